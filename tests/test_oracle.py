@@ -1,0 +1,293 @@
+"""Pins for the CPU oracle: closed forms, invariants, brute force and the
+hand-derived Top-p rows in tests/golden.  None of these re-types the
+oracle's own formula; each is chosen so that a dropped term, a wrong sign,
+scale or index, or a transposed operand in the oracle fails at least one.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import dsa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- pooling ----
+
+def test_block_bounds_ragged():
+    assert O.block_bounds(300, 128) == [(0, 128), (128, 256), (256, 300)]
+    assert O.block_bounds(256, 128) == [(0, 128), (128, 256)]
+    assert O.block_bounds(1, 64) == [(0, 1)]
+
+
+def test_pool_constant_blocks():
+    # a tensor constant inside each block pools to that constant
+    N, Bs, D = 300, 128, 5
+    vals = np.array([[1.5] * D, [-2.0] * D, [7.25] * D])
+    x = np.concatenate([np.tile(vals[i], (b - a, 1))
+                        for i, (a, b) in enumerate(O.block_bounds(N, Bs))])
+    np.testing.assert_array_equal(O.pool_blocks(x, Bs), vals)
+
+
+def test_pool_ramp_midpoint_ragged():
+    # x_t = t: the mean over [a, b) is (a + b - 1) / 2, also for the ragged tail
+    N, Bs = 300, 128
+    x = np.arange(N, dtype=np.float64)[:, None] * np.array([[1.0, -3.0]])
+    got = O.pool_blocks(x, Bs)
+    want = np.array([[(a + b - 1) / 2.0, -3.0 * (a + b - 1) / 2.0]
+                     for a, b in O.block_bounds(N, Bs)])
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------- block probs ----
+
+def test_probs_closed_form_log_weights():
+    # scale * qbar . kbar_j = log(j + 1)  ->  P_j = (j + 1) / sum
+    nB, scale = 6, 0.125
+    qbar = np.array([[1.0, 0.0]])
+    kbar = np.array([[math.log(j + 1) / scale, 3.0] for j in range(nB)])
+    P = O.block_probs(qbar, kbar, scale)
+    want = np.arange(1, nB + 1) / (nB * (nB + 1) / 2)
+    np.testing.assert_allclose(P[0], want, rtol=1e-13)
+
+
+def test_probs_rows_sum_to_one_and_shift_invariance():
+    rng = np.random.default_rng(0)
+    qbar, kbar = rng.normal(size=(9, 16)), rng.normal(size=(9, 16))
+    P = O.block_probs(qbar, kbar, 0.25)
+    assert np.all(np.abs(P.sum(1) - 1.0) <= 1e-12)
+    assert np.all(P >= 0)
+    # adding one vector to every key block adds a per-row constant to the logits
+    P2 = O.block_probs(qbar, kbar + rng.normal(size=(1, 16)), 0.25)
+    np.testing.assert_allclose(P, P2, rtol=1e-10)
+    # P is not symmetric in (q, k): swapping the operands must change it
+    assert not np.allclose(P, O.block_probs(kbar, qbar, 0.25))
+
+
+def test_probs_uniform_and_one_hot():
+    qbar = np.array([[1.0, 2.0]])
+    kbar = np.tile([[0.5, -1.0]], (5, 1))
+    np.testing.assert_allclose(O.block_probs(qbar, kbar, 1.0)[0], 0.2, rtol=1e-14)
+    kbar[3] = [1e3, 0.0]
+    P = O.block_probs(qbar, kbar, 1.0)[0]
+    assert P[3] == 1.0 and np.all(np.delete(P, 3) < 1e-300)
+
+
+def test_probs_reduced_renormalised():
+    nB, scale = 5, 1.0
+    qbar = np.array([[1.0]])
+    kbar = np.array([[math.log(j + 1)] for j in range(nB)])
+    P = O.block_probs(qbar, kbar, scale, cand=[np.array([1, 4])])[0]
+    np.testing.assert_allclose(P, [0, 2 / 7, 0, 0, 5 / 7], rtol=1e-14, atol=0)
+
+
+# ----------------------------------------------------------------- Top-p ----
+
+def _read_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "topp_rows.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            name, p, vals, cand, want = [t.strip() for t in line.split("|")]
+            r = np.array([float.fromhex(t) for t in vals.split()], np.float32)
+            cand = (None if cand == "*" else
+                    [] if cand == "-" else [int(t) for t in cand.split()])
+            want = [] if want == "-" else [int(t) for t in want.split()]
+            rows.append((name, float.fromhex(p), r, cand, want))
+    return rows
+
+
+@pytest.mark.parametrize("case", _read_golden(), ids=lambda c: c[0])
+def test_topp_golden_rows(case):
+    name, p, r, cand, want = case
+    assert list(O.topp_select_row(r, p, cand)) == want
+
+
+def _brute_force(r, p, cand):
+    """Smallest subset of cand reaching p in exact rational arithmetic, ties
+    between minimal subsets broken by the (score desc, index asc) order."""
+    from fractions import Fraction
+    vals = {j: Fraction(float(r[j])) for j in cand}
+    pf = Fraction(float(np.float32(p)))
+    if pf >= 1:
+        return sorted(cand)
+    rank = {j: n for n, j in enumerate(sorted(cand, key=lambda j: (-vals[j], j)))}
+    for size in range(1, len(cand) + 1):
+        hits = [s for s in itertools.combinations(cand, size)
+                if sum(vals[j] for j in s) >= pf]
+        if hits:
+            best = max(sum(vals[j] for j in s) for s in hits)
+            tops = [s for s in hits if sum(vals[j] for j in s) == best]
+            return sorted(min(tops, key=lambda s: sorted(rank[j] for j in s)))
+    return sorted(cand)
+
+
+def test_topp_brute_force_small_rows():
+    rng = np.random.default_rng(1)
+    for trial in range(300):
+        nB = int(rng.integers(1, 11))
+        z = rng.normal(scale=rng.uniform(0.1, 4.0), size=nB)
+        if trial % 5 == 0:          # plenty of exact ties
+            z = np.round(z)
+        r = (np.exp(z) / np.exp(z).sum()).astype(np.float32)
+        p = float(rng.choice([0.3, 0.5, 0.7, 0.9, 0.95, 0.99, 1.0]))
+        cand = list(range(nB))
+        if trial % 3 == 0:
+            cand = sorted(rng.choice(nB, size=int(rng.integers(0, nB + 1)),
+                                     replace=False).tolist())
+        got = list(O.topp_select_row(r, p, None if trial % 3 else cand))
+        assert got == _brute_force(r, p, cand), (r, p, cand)
+
+
+def test_topp_minimal_prefix_invariant():
+    rng = np.random.default_rng(2)
+    for _ in range(50):
+        nB = 40
+        z = rng.normal(scale=2.0, size=nB)
+        r = (np.exp(z) / np.exp(z).sum()).astype(np.float32)
+        p = float(rng.uniform(0.05, 0.99))
+        sel = O.topp_select_row(r, p)
+        tot = sum(float(r[j]) for j in sel)
+        assert tot >= float(np.float32(p)) or len(sel) == nB
+        # dropping the smallest kept block falls below p
+        smallest = min(sel, key=lambda j: (float(r[j]), -j))
+        assert tot - float(r[smallest]) < float(np.float32(p))
+        # nothing outside the set beats anything inside it
+        out = np.setdiff1d(np.arange(nB), sel)
+        if out.size:
+            assert r[out].max() <= r[sel].min()
+
+
+def test_topp_reduced_all_candidates_equals_full():
+    rng = np.random.default_rng(3)
+    P = rng.dirichlet(np.ones(23), size=30).astype(np.float32)
+    full = O.topp_select(P, 0.8)
+    rp = np.arange(31) * 23
+    cc = np.tile(np.arange(23), 30)
+    red = O.topp_select(P, 0.8, rp, cc)
+    np.testing.assert_array_equal(full[0], red[0])
+    np.testing.assert_array_equal(full[1], red[1])
+
+
+def test_topp_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        O.fp32_to_fixed(1.5)
+    with pytest.raises(ValueError):
+        O.fp32_to_fixed(-0.25)
+
+
+# ------------------------------------------------------------- attention ----
+
+def _qkv(N, D, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return (scale * rng.normal(size=(N, D)), scale * rng.normal(size=(N, D)),
+            rng.normal(size=(N, D)))
+
+
+def _all_blocks(nB):
+    return np.arange(nB + 1) * nB, np.tile(np.arange(nB), nB)
+
+
+@pytest.mark.parametrize("N,Bs", [(256, 64), (300, 128), (77, 32)])
+def test_attention_p1_equals_dense_textbook(N, Bs):
+    q, k, v = _qkv(N, 16, 4)
+    scale = 1 / 4.0
+    nB = (N + Bs - 1) // Bs
+    rp, col = _all_blocks(nB)
+    Os, lse, _ = O.sparse_attention_head(q, k, v, Bs, scale, rp, col)
+    Od, lsed = O.dense_attention(q, k, v, scale)
+    np.testing.assert_allclose(Os, Od, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lsed, rtol=1e-13)
+
+
+def test_attention_single_block_is_dense_on_that_block():
+    N, Bs, D = 300, 128, 8
+    q, k, v = _qkv(N, D, 5)
+    rp = np.array([0, 1, 2, 3])
+    col = np.array([2, 0, 1])          # block 0 -> 2 (ragged), 1 -> 0, 2 -> 1
+    Os, lse, _ = O.sparse_attention_head(q, k, v, Bs, 0.3, rp, col)
+    b = O.block_bounds(N, Bs)
+    for i, j in enumerate(col):
+        (a0, a1), (c0, c1) = b[i], b[j]
+        Od, ld = O.dense_attention(q[a0:a1], k[c0:c1], v[c0:c1], 0.3)
+        np.testing.assert_allclose(Os[a0:a1], Od, atol=1e-12)
+        np.testing.assert_allclose(lse[a0:a1], ld, rtol=1e-13)
+
+
+def test_attention_block_order_invariance():
+    N, Bs = 384, 64
+    q, k, v = _qkv(N, 8, 6)
+    nB = 6
+    rp = np.arange(nB + 1) * 3
+    col = np.array([0, 2, 5, 1, 3, 4, 0, 1, 2, 3, 4, 5, 5, 4, 3, 2, 1, 0])
+    col2 = col.reshape(nB, 3)[:, ::-1].reshape(-1)
+    A = O.sparse_attention_head(q, k, v, Bs, 0.5, rp, col)
+    B = O.sparse_attention_head(q, k, v, Bs, 0.5, rp, col2)
+    np.testing.assert_allclose(A[0], B[0], atol=1e-12)
+    np.testing.assert_allclose(A[1], B[1], rtol=1e-13)
+    np.testing.assert_allclose(A[2].reshape(nB, 3, Bs)[:, ::-1],
+                               B[2].reshape(nB, 3, Bs), rtol=1e-13)
+
+
+def test_attention_zero_query_closed_form():
+    # q = 0: every logit is 0, o_t = mean of the selected V rows and
+    # lse_t = log(#selected keys); block mass = |B_j| / sum |B_j'|
+    N, Bs, D = 200, 64, 4
+    _, k, v = _qkv(N, D, 7)
+    q = np.zeros((N, D))
+    rp = np.array([0, 2, 2, 3, 5])     # row 1 is empty
+    col = np.array([1, 3, 3, 0, 3])    # block 3 is ragged (8 tokens)
+    Os, lse, blk = O.sparse_attention_head(q, k, v, Bs, 1.0, rp, col)
+    b = O.block_bounds(N, Bs)
+    for i in range(4):
+        a0, a1 = b[i]
+        sel = col[rp[i]:rp[i + 1]]
+        if sel.size == 0:
+            assert np.all(Os[a0:a1] == 0) and np.all(lse[a0:a1] == -np.inf)
+            continue
+        keys = np.concatenate([np.arange(*b[j]) for j in sel])
+        np.testing.assert_allclose(Os[a0:a1], np.tile(v[keys].mean(0), (a1 - a0, 1)),
+                                   atol=1e-12)
+        np.testing.assert_allclose(lse[a0:a1], math.log(keys.size), rtol=1e-14)
+    M = O.block_mass(lse, blk, rp, N, Bs)
+    np.testing.assert_allclose(M, [64 / 72, 8 / 72, 1.0, 64 / 72, 8 / 72], rtol=1e-13)
+
+
+def test_block_mass_sums_to_one_and_matches_dense_weights():
+    N, Bs = 320, 64
+    q, k, v = _qkv(N, 8, 8, scale=0.8)
+    nB = 5
+    rp, col = _all_blocks(nB)
+    _, lse, blk = O.sparse_attention_head(q, k, v, Bs, 0.4, rp, col)
+    M = O.block_mass(lse, blk, rp, N, Bs).reshape(nB, nB)
+    np.testing.assert_allclose(M.sum(1), 1.0, rtol=1e-12)
+    # at p = 1 the mass equals the block sums of the dense softmax matrix
+    z = 0.4 * q @ k.T
+    w = np.exp(z) / np.exp(z).sum(1, keepdims=True)
+    b = O.block_bounds(N, Bs)
+    dense = np.array([[w[a0:a1, c0:c1].sum(1).mean() for (c0, c1) in b] for (a0, a1) in b])
+    np.testing.assert_allclose(M, dense, rtol=1e-12)
+
+
+def test_recall_is_one_at_p1_and_pipeline_reduced_equals_full():
+    N, Bs, D = 256, 64, 8
+    q, k, v = _qkv(N, D, 9, scale=1.5)
+    nB = 4
+    rp, col = _all_blocks(nB)
+    np.testing.assert_allclose(O.recall(q, k, Bs, 0.35, rp, col), 1.0, rtol=1e-12)
+    full = O.pipeline_head(q, k, v, Bs, 0.35, 0.9)
+    red = O.pipeline_head(q, k, v, Bs, 0.35, 0.9, rp, col)
+    np.testing.assert_array_equal(full["row_ptr"], red["row_ptr"])
+    np.testing.assert_array_equal(full["col"], red["col"])
+    np.testing.assert_array_equal(full["O"], red["O"])
+
+
+def test_executed_flops_counts_ragged_blocks():
+    rp = np.array([0, 2, 3])
+    col = np.array([0, 1, 1])          # N = 100, Bs = 64: blocks of 64 and 36
+    assert O.executed_flops(rp, col, 100, 64, 8) == 4 * 8 * (64 * 64 + 64 * 36 + 36 * 36)
