@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the dynamic block-sparse attention pipeline on B200.
+
+One step = the whole path on one batch: pooled block scores + row softmax
+(dsa_pool_score), Top-p selection to CSR (dsa_select_topp), block-sparse
+attention forward (dsa_attn_fwd) and exact block mass (dsa_block_mass), on
+seeded synthetic Q/K/V already resident in HBM.
+
+Metric: executed attention TFLOP/s, 4 * sum over selected (i, j) of
+|B_i| |B_j| D, divided by the whole step's device time; the attention kernel
+alone is reported against the measured bf16 tensor peak, and the step is
+compared with a dense p = 1 run of the same kernel (all blocks selected).
+
+Multi-GPU (torchrun): every rank runs its own batch (seed + rank), with no
+collective on the data path; the JSON value is the sum of executed FLOPs
+over the max step time across ranks ("weak" scaling).
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from dynamic_block_sparse_pool_b200 import ops, synth  # noqa: E402
+
+METRIC = "block-sparse attn fwd TFLOP/s (executed) & % bf16 peak; speedup vs p=1"
+LAUNCHES_PER_STEP = 7  # pool_means, block_scores, select, csr_scan, compact, attn_fwd, block_mass
+ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn_sm100.cu")
+# DRAM bytes per attention launch from an ncu capture, keyed by the sha256
+# prefix of attn_sm100.cu at capture time (scaled to the full workload when
+# the capture ran a smaller case); stale entries are ignored.
+ATTN_TRAFFIC = {}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("dsa", "reference"), default="dsa")
+    ap.add_argument("--workload", default=synth.WAN21.name, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--p", type=float, default=0.9)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-dense", action="store_true", help="skip the p=1 reference run")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------- utils --
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(bf16_burst=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    hbm=float(d["hbm_gbs"]), source="measured")
+    return dict(bf16_burst=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def attn_source_hash():
+    with open(ATTN_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def executed_flops(row_ptr, col_idx, N, block, D, nB):
+    """4 * D * sum over selected (row, col) of |B_row| * |B_col| (exact, int64)."""
+    sizes = torch.full((nB,), block, dtype=torch.int64, device=row_ptr.device)
+    sizes[-1] = N - (nB - 1) * block
+    rp = row_ptr.long()
+    nnz = int(rp[-1])
+    counts = rp[1:] - rp[:-1]
+    rows = torch.arange(counts.numel(), device=rp.device)
+    qs = sizes[rows % nB]
+    ks = sizes[col_idx[:nnz].long()]
+    per_row = torch.zeros(counts.numel(), dtype=torch.int64, device=rp.device)
+    per_row.index_add_(0, torch.repeat_interleave(rows, counts), ks)
+    return int(4 * D * (qs * per_row).sum().item()), nnz
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.uuid = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [[c.strip() for c in line.split(",")] for line in out.splitlines() if line.strip()]
+        if self.uuid:
+            mine = [r for r in rows if len(r) > 1 and r[1] == self.uuid]
+            rows = mine or rows
+        if not rows:
+            return None
+        try:
+            sm = [float(r[2]) for r in rows]
+            mx = max(float(r[3]) for r in rows)
+            pw = [float(r[4]) for r in rows]
+        except (ValueError, IndexError):
+            return None
+        thr = 0.5 * max(pw)
+        load = [r for r, p in zip(rows, pw) if p >= thr] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in load for n, v in zip(names, r[6:10]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(float(r[2]) for r in load), "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(pw)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------- oracle sample --
+
+def oracle_sample(w, q, k, v, p, seconds, head=0):
+    """Time the CPU oracle on one head: its own pooled scores, softmax and
+    Top-p for every row, then attention + block mass for query-block rows
+    spread over the head until about `seconds` of CPU time is spent.
+    Returns (tflops, description, threads)."""
+    import numpy as np
+    from oracle import dsa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+    qh, kh, vh = f64(q[0, head]), f64(k[0, head]), f64(v[0, head])
+    scale = 1.0 / math.sqrt(w.head_dim)
+    nB = w.n_blocks
+    t0 = time.perf_counter()
+    P = O.block_probs(O.pool_blocks(qh, w.block), O.pool_blocks(kh, w.block), scale)
+    rp, col = O.topp_select(P.astype(np.float32), p)
+    t_search = time.perf_counter() - t0
+    order = list(range(0, nB, max(1, nB // 64))) + [nB - 1]
+    seen, rows, flops = set(), [], 0
+    t_attn = 0.0
+    for i in order:
+        if i in seen:
+            continue
+        seen.add(i)
+        t1 = time.perf_counter()
+        Oo, lo, blk = O.sparse_attention_head(qh, kh, vh, w.block, scale, rp, col, rows=[i])
+        O.block_mass(lo, blk, rp, w.N, w.block)
+        t_attn += time.perf_counter() - t1
+        a, b = i * w.block, min(w.N, (i + 1) * w.block)
+        flops += sum(4 * w.head_dim * (b - a) * (min(w.N, (j + 1) * w.block) - j * w.block)
+                     for j in col[rp[i]:rp[i + 1]])
+        rows.append(i)
+        if t_attn + t_search >= seconds:
+            break
+    t_total = t_attn + t_search * len(rows) / nB
+    desc = (f"oracle (NumPy fp64) on head {head} of {w.name}: pooled scores, softmax and "
+            f"exact Top-p for all {nB} rows ({t_search:.2f} s, pro-rated), then attention on "
+            f"{len(rows)} of {nB} query-block rows ({t_attn:.2f} s); "
+            f"{flops / 1e9:.1f} GFLOP executed")
+    return flops / t_total / 1e12, desc, threads, t_total
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    q, k, v = synth.make_qkv(w, args.seed, heads=[0])
+    per_step = max(1.0, args.cpu_seconds / 4)
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, args.p, per_step / 4)
+    vals, times = [], []
+    desc, threads = "", 1
+    for _ in range(args.steps):
+        val, desc, threads, t = oracle_sample(w, q, k, v, args.p, per_step)
+        vals.append(val)
+        times.append(t)
+    value = sum(vals) / len(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w.describe(), "p": args.p, "seed": args.seed,
+            "batch": w.batch, "heads": w.heads, "tokens": w.N, "head_dim": w.head_dim,
+            "block": w.block, "grid": [w.T, w.Hg, w.W], "parallelism": f"replicas{args.gpus}",
+            "l2": "inputs larger than L2 (Q,K,V %.2f GB)" % (3 * w.BH * w.N * w.head_dim * 2 / 1e9)}
+
+
+# ---------------------------------------------------------------- GPU bench --
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+    nB = w.n_blocks
+    rows = B * H * nB
+    scale = 1.0 / math.sqrt(D)
+    q_c, k_c, v_c = synth.make_qkv(w, args.seed + rank)
+    q, k, v = q_c.to(dev), k_c.to(dev), v_c.to(dev)
+
+    P = torch.empty(B * H, nB, nB, device=dev, dtype=torch.float32)
+    ws_pool = torch.empty(ops.workspace_size(0, B, H, N, D, blk), device=dev, dtype=torch.uint8)
+    ws_sel = torch.empty(ops.workspace_size(1, B, H, N, D, blk), device=dev, dtype=torch.uint8)
+    row_ptr = torch.empty(rows + 1, device=dev, dtype=torch.int32)
+    col_idx = torch.empty(rows * nB, device=dev, dtype=torch.int32)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, N, device=dev, dtype=torch.float32)
+    blk_lse = torch.empty(rows * nB, blk, device=dev, dtype=torch.float32)
+    mass = torch.empty(rows * nB, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def search():
+        ops.pool_score(q, k, blk, scale, out=P, workspace=ws_pool)
+        ops.select_topp(P, args.p, row_ptr=row_ptr, col_idx=col_idx, workspace=ws_sel)
+
+    def attend(rp=row_ptr, ci=col_idx):
+        ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=blk_lse)
+
+    def finish(rp=row_ptr):
+        ops.block_mass(lse, blk_lse, rp, blk, mass=mass)
+
+    # one untimed pass for the mask statistics
+    search(); attend(); finish()
+    ops.device_status(dev)
+    flops, nnz = executed_flops(row_ptr, col_idx, N, blk, D, nB)
+    dense_flops = 4 * D * B * H * N * N
+    for _ in range(args.warmup):
+        search(); attend(); finish()
+    torch.cuda.synchronize(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for s in range(args.steps):
+        e = ev[s]
+        e[0].record(stream); search()
+        e[1].record(stream); attend()
+        e[2].record(stream); finish()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(world)
+    ops.device_status(dev)
+    t_step = [e[0].elapsed_time(e[3]) for e in ev]
+    t_search = [e[0].elapsed_time(e[1]) for e in ev]
+    t_attn = [e[1].elapsed_time(e[2]) for e in ev]
+    t_mass = [e[2].elapsed_time(e[3]) for e in ev]
+    ms_step = reduce_max(sum(t_step) / len(t_step), world)
+    ms_attn = sum(t_attn) / len(t_attn)
+    total_flops = reduce_sum(float(flops), world)
+    value = total_flops / (ms_step * 1e-3) / 1e12
+    attn_tflops = flops / (ms_attn * 1e-3) / 1e12
+    peaks = measured_peaks()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": config_of(w, args),
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+    }
+    traffic = ATTN_TRAFFIC.get(attn_source_hash())
+    line["roofline"] = {
+        "bound": "tensor", "kernel": "attn_fwd_sm100_kernel", "achieved": attn_tflops,
+        "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+        "frac": attn_tflops / peaks["bf16_sustained"],
+        "peak_kind": f"{peaks['source']} bf16 sustained (kernel timed inside multi-second step loop)",
+        "frac_of_burst_peak": attn_tflops / peaks["bf16_burst"],
+        "traffic": traffic,
+        "algorithmic_flop_per_launch": flops,
+    }
+    line["breakdown_ms"] = {"search": sum(t_search) / len(t_search), "attn": ms_attn,
+                            "mass": sum(t_mass) / len(t_mass)}
+    line["mask"] = {"nnz_blocks": nnz, "density": nnz / (rows * nB),
+                    "executed_tflop": flops / 1e12, "dense_tflop": dense_flops / 1e12}
+    line["clocks"] = clk
+
+    # dense p = 1 reference: the same kernel over an all-blocks CSR
+    if not args.no_dense:
+        rp_all = (torch.arange(rows + 1, device=dev, dtype=torch.int64) * nB).to(torch.int32)
+        col_all = torch.arange(nB, device=dev, dtype=torch.int32).repeat(rows)
+        attend(rp_all, col_all)
+        torch.cuda.synchronize(dev)
+        kd = max(2, args.steps // 3)
+        ed = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(kd)]
+        for e in ed:
+            e[0].record(stream); attend(rp_all, col_all); e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms_dense = sum(e[0].elapsed_time(e[1]) for e in ed) / kd
+        red = dense_flops / flops
+        line["speedup_vs_p1"] = {
+            "dense_attn_ms": ms_dense,
+            "dense_attn_tflops": dense_flops / (ms_dense * 1e-3) / 1e12,
+            "attn_only": ms_dense / ms_attn,
+            "pipeline": ms_dense / (sum(t_step) / len(t_step)),
+            "executed_flop_reduction": red,
+            "pipeline_over_reduction": ms_dense / (sum(t_step) / len(t_step)) / red,
+        }
+        del rp_all, col_all
+
+    # end to end through the public calls with pinned host buffers
+    if not args.no_e2e:
+        qh, kh, vh = q_c.pin_memory(), k_c.pin_memory(), v_c.pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        ke = max(2, args.steps // 2)
+        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(ke + 1)]
+        for s in range(ke + 1):  # first iteration is a warm-up
+            ee[s][0].record(stream)
+            q.copy_(qh, non_blocking=True); k.copy_(kh, non_blocking=True); v.copy_(vh, non_blocking=True)
+            search(); attend(); finish()
+            oh.copy_(out, non_blocking=True)
+            ee[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ee[1:]) / ke, world)
+        line["e2e"] = {"value": total_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "ms_per_step": ms_e2e,
+                       "h2d_bytes_per_step": 3 * q_c.numel() * q_c.element_size(),
+                       "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        val, desc, threads, _ = oracle_sample(w, q_c, k_c, v_c, args.p, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

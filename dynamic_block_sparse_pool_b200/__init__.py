@@ -3,7 +3,14 @@
 Pipeline per (batch, head): mean-pooled block scores with a row softmax,
 per-row Top-p block selection (optionally restricted to a candidate set),
 exact block-sparse attention over the selected blocks, and the exact softmax
-mass of every selected block.  All arithmetic runs in ``libdsa.so``; this
-package only marshals arguments to it.
+mass of every selected block.  All arithmetic runs in ``libdsa.so``; the
+Python layer only marshals arguments (see ``ops``).  The library is loaded
+on the first call, and a call fails loudly if it has not been built.
 """
-__all__ = ["synth"]
+from . import ops, synth  # noqa: F401
+from ._lib import DSAError  # noqa: F401
+from .ops import (attn_fwd, block_mass, device_status, pool_score,  # noqa: F401
+                  select_topp, sparse_attention)
+
+__all__ = ["ops", "synth", "DSAError", "pool_score", "select_topp", "attn_fwd",
+           "block_mass", "sparse_attention", "device_status"]

@@ -1,0 +1,66 @@
+// Exact softmax mass of every selected key block.
+//
+// GSRS (arXiv 2610.21129), abstract: the exact attention weight of each
+// block comes out of the FlashAttention pass at negligible overhead; Figure
+// 2 measures the recall of a block mask with the same quantity.
+//
+// mass[s] = mean over the queries t of block i of exp(blk_lse[s, t] - lse_t),
+// where blk_lse[s, t] is the log of the block's share of the softmax
+// denominator and lse_t the log of the whole denominator (both written by
+// the attention kernel).  One warp per CSR row keeps the row's lse values in
+// registers and reads each slot's block-size run of blk_lse once, coalesced.
+#include "common.cuh"
+
+namespace dsa {
+namespace {
+
+template <int BS>
+__global__ void __launch_bounds__(256)
+block_mass_kernel(const float* __restrict__ lse, const float* __restrict__ blk, int N,
+                  int nB, int rows, const int32_t* __restrict__ row_ptr,
+                  float* __restrict__ mass) {
+  constexpr int PER = BS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= rows) return;
+  const int bh = r / nB, i = r - bh * nB;
+  const int q0 = i * BS;
+  const int qlen = min(BS, N - q0);
+  float lv[PER];
+#pragma unroll
+  for (int m = 0; m < PER; ++m) {
+    const int t = lane + 32 * m;
+    lv[m] = t < qlen ? lse[(size_t)bh * N + q0 + t] : 0.f;
+  }
+  const float inv = 1.0f / (float)qlen;
+  const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
+  for (int s = s0; s < s1; ++s) {
+    const float* b = blk + (size_t)s * BS;
+    float acc = 0.f;
+#pragma unroll
+    for (int m = 0; m < PER; ++m) {
+      const int t = lane + 32 * m;
+      if (t < qlen) acc += expf(b[t] - lv[m]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) mass[s] = acc * inv;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
+                              int block, const int32_t* row_ptr, float* mass,
+                              cudaStream_t s) {
+  const int nB = ceil_div(N, block);
+  const int rows = BH * nB;
+  const int grid = ceil_div(rows, 8);
+  if (block == 64)
+    block_mass_kernel<64><<<grid, 256, 0, s>>>(lse, blk_lse, N, nB, rows, row_ptr, mass);
+  else
+    block_mass_kernel<128><<<grid, 256, 0, s>>>(lse, blk_lse, N, nB, rows, row_ptr, mass);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

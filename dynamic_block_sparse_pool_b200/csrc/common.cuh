@@ -1,0 +1,62 @@
+// Shared definitions for the libdsa kernels (device side and launchers).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace dsa {
+
+// Bits of the device-side error word (see dsa_device_status).
+enum : unsigned {
+  kErrCsrIndex = 1u,     // a CSR column index outside [0, nB)
+  kErrRowPtr = 2u,       // a row_ptr entry that is negative or decreasing
+  kErrProb = 4u,         // a probability outside [0, 1] or NaN
+  kErrTimeout = 8u,      // a bounded wait on an mbarrier ran out
+};
+
+// Upper bound for one mbarrier wait before a kernel gives up (nanoseconds).
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+__device__ __forceinline__ void flag_error(unsigned* err, unsigned bits) {
+  if (err) atomicOr(err, bits);
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float x) { return x; }
+  static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Launchers (one per kernel family); all return the launch error.
+cudaError_t launch_pool_means(const void* q, const void* k, bool bf16, int BH, int N,
+                              int D, int block, float* qbar, float* kbar,
+                              cudaStream_t s);
+cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, int nB,
+                                int D, float scale, const int32_t* cand_row_ptr,
+                                const int32_t* cand_col, float* probs, unsigned* err,
+                                cudaStream_t s);
+cudaError_t launch_select(const float* probs, int rows, int nB, float p,
+                          const int32_t* cand_row_ptr, const int32_t* cand_col,
+                          int32_t* row_ptr, int32_t* col_idx, uint32_t* bitmaps,
+                          int32_t* counts, unsigned* err, cudaStream_t s);
+cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, bool bf16,
+                             int BH, int N, int D, int block, float scale,
+                             const int32_t* row_ptr, const int32_t* col_idx, void* out,
+                             float* lse, float* blk_lse, unsigned* err, cudaStream_t s);
+cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int BH,
+                              int N, int D, float scale, const int32_t* row_ptr,
+                              const int32_t* col_idx, void* out, float* lse,
+                              float* blk_lse, unsigned* err, cudaStream_t s,
+                              const char** why);
+cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
+                              int block, const int32_t* row_ptr, float* mass,
+                              cudaStream_t s);
+
+}  // namespace dsa

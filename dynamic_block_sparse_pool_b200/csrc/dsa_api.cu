@@ -1,0 +1,245 @@
+// C ABI of libdsa (declared in include/dsa.h): argument checks, error
+// reporting and dispatch to the kernel launchers.  No call allocates device
+// memory or synchronises the host, except dsa_device_status.
+#include <climits>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "dsa.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// Device-side error word shared by all kernels of the library.
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+dsa_status fail(dsa_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+dsa_status fail(dsa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+dsa_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(DSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  unsigned* err_word = nullptr;
+};
+
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+// Per-device set-up: architecture check and the error word's address.
+dsa_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device id %d", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.sm100 = (major == 10 && minor == 0);
+    if (d.sm100) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_device_error);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+      d.err_word = static_cast<unsigned*>(p);
+    }
+    d.init = true;
+  }
+  if (!d.sm100)
+    return fail(DSA_ERR_UNSUPPORTED, "libdsa is built for sm_100a (B200); device %d is not", dev);
+  *out = &d;
+  return DSA_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by the tensor-level calls.
+dsa_status check_shape(int B, int H, int N, int D, int block) {
+  if (B < 1 || H < 1 || N < 1) return fail(DSA_ERR_INVALID_ARG, "B, H, N must be >= 1 (got %d, %d, %d)", B, H, N);
+  if ((long long)B * H > 65535) return fail(DSA_ERR_INVALID_ARG, "B*H = %lld exceeds 65535", (long long)B * H);
+  if (D != 64 && D != 128) return fail(DSA_ERR_INVALID_ARG, "head_dim D must be 64 or 128 (got %d)", D);
+  if (block != 64 && block != 128) return fail(DSA_ERR_INVALID_ARG, "block must be 64 or 128 (got %d)", block);
+  const long long nB = (N + (long long)block - 1) / block;
+  if ((long long)B * H * nB >= INT_MAX) return fail(DSA_ERR_INVALID_ARG, "too many block rows");
+  return DSA_OK;
+}
+
+dsa_status check_blocks_limit(long long rows, int nB) {
+  if (nB < 1 || nB > DSA_MAX_BLOCKS)
+    return fail(DSA_ERR_INVALID_ARG, "nB = %d blocks per row; supported 1..%d", nB, DSA_MAX_BLOCKS);
+  if (rows * nB >= INT_MAX) return fail(DSA_ERR_INVALID_ARG, "rows * nB exceeds the int32 CSR range");
+  return DSA_OK;
+}
+
+bool cand_ok(const int32_t* rp, const int32_t* col) { return (rp == nullptr) == (col == nullptr); }
+
+size_t pool_ws_bytes(long long BH, long long nB, int D) { return (size_t)(2 * BH * nB * D) * sizeof(float); }
+size_t select_ws_bytes(long long rows) { return (size_t)(rows * 33) * sizeof(uint32_t); }
+
+}  // namespace
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+const char* dsa_last_error(void) { return g_last_error.c_str(); }
+
+size_t dsa_workspace_size(int op, int B, int H, int N, int D, int block) {
+  if (check_shape(B, H, N, D, block) != DSA_OK) return 0;
+  const long long nB = (N + (long long)block - 1) / block;
+  const long long BH = (long long)B * H;
+  if (op == DSA_OP_POOL_SCORE) return pool_ws_bytes(BH, nB, D);
+  if (op == DSA_OP_SELECT_TOPP) return select_ws_bytes(BH * nB);
+  return 0;
+}
+
+dsa_status dsa_pool_score(const void* q, const void* k, dsa_dtype dt, int B, int H, int N,
+                          int D, int block, float scale, const int32_t* cand_row_ptr,
+                          const int32_t* cand_col, float* probs, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !probs || !workspace) return fail(DSA_ERR_INVALID_ARG, "null q, k, probs or workspace");
+  if (dt != DSA_F32 && dt != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  dsa_status st = check_shape(B, H, N, D, block);
+  if (st != DSA_OK) return st;
+  const int nB = (N + block - 1) / block;
+  const long long BH = (long long)B * H;
+  if ((st = check_blocks_limit(BH * nB, nB)) != DSA_OK) return st;
+  if (!cand_ok(cand_row_ptr, cand_col)) return fail(DSA_ERR_INVALID_ARG, "cand_row_ptr and cand_col must both be set or both be NULL");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(probs, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q, k and workspace must be 16-byte aligned, probs 4-byte aligned");
+  if (ws_bytes < pool_ws_bytes(BH, nB, D))
+    return fail(DSA_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes, pool_ws_bytes(BH, nB, D));
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* qbar = static_cast<float*>(workspace);
+  float* kbar = qbar + BH * nB * D;
+  cudaError_t e = dsa::launch_pool_means(q, k, dt == DSA_BF16, (int)BH, N, D, block, qbar, kbar, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pool_means launch");
+  e = dsa::launch_block_scores(qbar, kbar, (int)BH, nB, D, scale, cand_row_ptr, cand_col, probs,
+                               dev->err_word, s);
+  if (e != cudaSuccess) return cuda_fail(e, "block_scores launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_select_topp(const float* probs, int rows, int nB, float p,
+                           const int32_t* cand_row_ptr, const int32_t* cand_col,
+                           int32_t* row_ptr, int32_t* col_idx, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (!probs || !row_ptr || !col_idx || !workspace)
+    return fail(DSA_ERR_INVALID_ARG, "null probs, row_ptr, col_idx or workspace");
+  if (rows < 1) return fail(DSA_ERR_INVALID_ARG, "rows must be >= 1 (got %d)", rows);
+  dsa_status st = check_blocks_limit(rows, nB);
+  if (st != DSA_OK) return st;
+  if (!(p > 0.f && p <= 1.f)) return fail(DSA_ERR_INVALID_ARG, "p must be in (0, 1] (got %g)", (double)p);
+  if (!cand_ok(cand_row_ptr, cand_col)) return fail(DSA_ERR_INVALID_ARG, "cand_row_ptr and cand_col must both be set or both be NULL");
+  if (!aligned(probs, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(workspace, 16))
+    return fail(DSA_ERR_INVALID_ARG, "misaligned pointer");
+  if (ws_bytes < select_ws_bytes(rows))
+    return fail(DSA_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes, select_ws_bytes(rows));
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  uint32_t* bitmaps = static_cast<uint32_t*>(workspace);
+  int32_t* counts = reinterpret_cast<int32_t*>(bitmaps + (size_t)rows * 32);
+  cudaError_t e = dsa::launch_select(probs, rows, nB, p, cand_row_ptr, cand_col, row_ptr, col_idx,
+                                     bitmaps, counts, dev->err_word, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select_topp launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype dt, int B, int H,
+                        int N, int D, int block, float scale, const int32_t* row_ptr,
+                        const int32_t* col_idx, void* out, float* lse, float* blk_lse,
+                        void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !out || !row_ptr || !col_idx)
+    return fail(DSA_ERR_INVALID_ARG, "null q, k, v, out, row_ptr or col_idx");
+  if (dt != DSA_F32 && dt != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  dsa_status st = check_shape(B, H, N, D, block);
+  if (st != DSA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(lse, 4) || !aligned(blk_lse, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned; index and float arrays 4-byte aligned");
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  cudaError_t e;
+  if (dt == DSA_BF16 && block == 128 && N >= 128) {
+    const char* why = nullptr;
+    e = dsa::launch_attn_sm100(q, k, v, BH, N, D, scale, row_ptr, col_idx, out, lse, blk_lse,
+                               dev->err_word, s, &why);
+    if (e != cudaSuccess && why) return fail(DSA_ERR_CUDA, "attn_fwd: %s", why);
+  } else {
+    e = dsa::launch_attn_simt(q, k, v, dt == DSA_BF16, BH, N, D, block, scale, row_ptr, col_idx,
+                              out, lse, blk_lse, dev->err_word, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_block_mass(const float* lse, const float* blk_lse, int B, int H, int N, int block,
+                          const int32_t* row_ptr, float* mass, void* stream) {
+  g_last_error.clear();
+  if (!lse || !blk_lse || !row_ptr || !mass)
+    return fail(DSA_ERR_INVALID_ARG, "null lse, blk_lse, row_ptr or mass");
+  dsa_status st = check_shape(B, H, N, 64, block);
+  if (st != DSA_OK) return st;
+  if (!aligned(lse, 4) || !aligned(blk_lse, 4) || !aligned(row_ptr, 4) || !aligned(mass, 4))
+    return fail(DSA_ERR_INVALID_ARG, "misaligned pointer");
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  cudaError_t e = dsa::launch_block_mass(lse, blk_lse, B * H, N, block, row_ptr, mass,
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block_mass launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_device_status(void* stream) {
+  g_last_error.clear();
+  DeviceInfo* dev = nullptr;
+  dsa_status st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (word == 0) return DSA_OK;
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s", word,
+              (word & dsa::kErrCsrIndex) ? " csr-index-out-of-range" : "",
+              (word & dsa::kErrRowPtr) ? " bad-row-ptr" : "",
+              (word & dsa::kErrProb) ? " probability-outside-[0,1]" : "",
+              (word & dsa::kErrTimeout) ? " wait-timeout" : "");
+}
+
+}  // extern "C"

@@ -1,0 +1,175 @@
+"""PyTorch-facing calls of libdsa.
+
+PyTorch supplies device memory and the current CUDA stream; every step of
+the computation runs in libdsa's kernels.  Tensors are [B, H, N, D],
+contiguous, bf16 or fp32, on one CUDA device.
+"""
+from __future__ import annotations
+
+import math
+from typing import NamedTuple, Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import check, lib
+
+Csr = Tuple[torch.Tensor, torch.Tensor]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(t: torch.Tensor):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _lib.DSA_BF16
+    if t.dtype == torch.float32:
+        return _lib.DSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _check_qkv(*ts: torch.Tensor):
+    t0 = ts[0]
+    if t0.dim() != 4:
+        raise ValueError("expected [B, H, N, D] tensors")
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+        if t.shape != t0.shape or t.dtype != t0.dtype or t.device != t0.device:
+            raise ValueError("q, k, v must share shape, dtype and device")
+    return t0.shape
+
+
+def _check_csr(csr: Optional[Csr], rows: int):
+    if csr is None:
+        return None, None
+    rp, col = csr
+    for t in (rp, col):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("CSR tensors must be contiguous int32 CUDA tensors")
+    if rp.numel() != rows + 1:
+        raise ValueError(f"row_ptr must have {rows + 1} entries, got {rp.numel()}")
+    return rp, col
+
+
+def n_blocks(N: int, block: int) -> int:
+    return (N + block - 1) // block
+
+
+def workspace_size(op: int, B: int, H: int, N: int, D: int, block: int) -> int:
+    return int(lib().dsa_workspace_size(op, B, H, N, D, block))
+
+
+def pool_score(q: torch.Tensor, k: torch.Tensor, block: int, scale: Optional[float] = None,
+               cand: Optional[Csr] = None, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """P [B*H, nB, nB] fp32: row softmax of scale * (block means of Q).(block means of K)."""
+    B, H, N, D = _check_qkv(q, k)
+    nB = n_blocks(N, block)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    crp, ccol = _check_csr(cand, B * H * nB)
+    if out is None:
+        out = torch.empty(B * H, nB, nB, device=q.device, dtype=torch.float32)
+    ws_bytes = workspace_size(_lib.DSA_OP_POOL_SCORE, B, H, N, D, block)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
+    st = lib().dsa_pool_score(q.data_ptr(), k.data_ptr(), _dtype_code(q), B, H, N, D, block,
+                              scale, _ptr(crp), _ptr(ccol), out.data_ptr(), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream(q))
+    check(st, "dsa_pool_score")
+    return out
+
+
+def select_topp(probs: torch.Tensor, p: float, cand: Optional[Csr] = None,
+                row_ptr: Optional[torch.Tensor] = None, col_idx: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None) -> Csr:
+    """CSR (row_ptr [rows+1], col_idx [capacity rows*nB]) of the Top-p block sets."""
+    if probs.dtype != torch.float32 or not probs.is_cuda or not probs.is_contiguous():
+        raise ValueError("probs must be a contiguous fp32 CUDA tensor")
+    nB = probs.shape[-1]
+    rows = probs.numel() // nB
+    crp, ccol = _check_csr(cand, rows)
+    dev = probs.device
+    if row_ptr is None:
+        row_ptr = torch.empty(rows + 1, device=dev, dtype=torch.int32)
+    if col_idx is None:
+        col_idx = torch.empty(rows * nB, device=dev, dtype=torch.int32)
+    ws_bytes = rows * 33 * 4
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    st = lib().dsa_select_topp(probs.data_ptr(), rows, nB, float(p), _ptr(crp), _ptr(ccol),
+                               row_ptr.data_ptr(), col_idx.data_ptr(), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream(probs))
+    check(st, "dsa_select_topp")
+    return row_ptr, col_idx
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.Tensor,
+             col_idx: torch.Tensor, block: int, scale: Optional[float] = None,
+             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             blk_lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+             want_blk_lse: bool = True):
+    """(O [B,H,N,D], lse [B,H,N] or None, blk_lse [nnz, block] or None).
+
+    When blk_lse is wanted but not given, nnz is read from row_ptr (one
+    device-to-host copy)."""
+    B, H, N, D = _check_qkv(q, k, v)
+    nB = n_blocks(N, block)
+    _check_csr((row_ptr, col_idx), B * H * nB)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32)
+    if want_blk_lse and blk_lse is None:
+        nnz = int(row_ptr[-1].item())
+        blk_lse = torch.empty(max(nnz, 1), block, device=q.device, dtype=torch.float32)
+    st = lib().dsa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, N, D,
+                            block, scale, row_ptr.data_ptr(), col_idx.data_ptr(), out.data_ptr(),
+                            _ptr(lse), _ptr(blk_lse), _stream(q))
+    check(st, "dsa_attn_fwd")
+    return out, lse, blk_lse
+
+
+def block_mass(lse: torch.Tensor, blk_lse: torch.Tensor, row_ptr: torch.Tensor, block: int,
+               mass: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """mass [nnz] (capacity blk_lse.shape[0]): exact softmax mass of each selected block."""
+    B, H, N = lse.shape
+    if mass is None:
+        mass = torch.empty(blk_lse.shape[0], device=lse.device, dtype=torch.float32)
+    st = lib().dsa_block_mass(lse.data_ptr(), blk_lse.data_ptr(), B, H, N, block,
+                              row_ptr.data_ptr(), mass.data_ptr(), _stream(lse))
+    check(st, "dsa_block_mass")
+    return mass
+
+
+def device_status(device: Optional[torch.device] = None) -> None:
+    """Synchronises the current stream and raises DSAError if a kernel flagged bad input."""
+    s = torch.cuda.current_stream(device).cuda_stream
+    check(lib().dsa_device_status(s), "dsa_device_status")
+
+
+class SparseAttention(NamedTuple):
+    out: torch.Tensor          # [B, H, N, D]
+    lse: torch.Tensor          # [B, H, N]
+    probs: torch.Tensor        # [B*H, nB, nB]
+    row_ptr: torch.Tensor      # [B*H*nB + 1]
+    col_idx: torch.Tensor      # [nnz]
+    mass: torch.Tensor         # [nnz]
+
+
+def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: float,
+                     block: int = 128, scale: Optional[float] = None,
+                     cand: Optional[Csr] = None) -> SparseAttention:
+    """Whole pipeline: pooled scores -> Top-p selection -> sparse attention -> block mass."""
+    probs = pool_score(q, k, block, scale, cand)
+    row_ptr, col_idx = select_topp(probs, p, cand)
+    out, lse, blk = attn_fwd(q, k, v, row_ptr, col_idx, block, scale)
+    mass = block_mass(lse, blk, row_ptr, block)
+    nnz = blk.shape[0] if int(row_ptr[-1].item()) > 0 else 0
+    return SparseAttention(out, lse, probs, row_ptr, col_idx[:nnz], mass[:nnz])

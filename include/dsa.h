@@ -1,0 +1,190 @@
+/*
+ * dsa.h -- C ABI of libdsa: dynamic block-sparse self-attention for video
+ * diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * The pipeline, per (batch b, head h), over N tokens cut into nB = ceil(N /
+ * block) blocks B_i = [i*block, min(N, (i+1)*block)):
+ *
+ *   dsa_pool_score   qbar_i, kbar_j = means of the rows of Q, K in each block;
+ *                    P_ij = softmax_j(scale * qbar_i . kbar_j), over all key
+ *                    blocks or over a candidate set C_i (reduced search).
+ *   dsa_select_topp  per row i: the shortest prefix of the candidates ordered
+ *                    by (P desc, block index asc) whose mass is >= p, as CSR.
+ *   dsa_attn_fwd     exact softmax attention of every query in B_i over the
+ *                    keys of the selected blocks, with per-block log-sums.
+ *   dsa_block_mass   the exact softmax mass each selected block receives.
+ *
+ * Sources: "Sparse Attention for Video Generation Acceleration via Growing
+ * Sparsity and Reduced Search" (GSRS, arXiv 2610.21129): abstract (Top-p
+ * selection; exact attention weights inside the FlashAttention pass; reduced
+ * search over an early candidate set), Figure 3 (block-level attention maps)
+ * and Figure 4 (growing Top-p, reduced search, mask reuse).  "DSV" (arXiv
+ * 2502.07590) abstract: kernels that identify critical key blocks and then
+ * compute the sparse attention.  The mean-pooled block score is the method's
+ * cheap estimator of the block-level map; the papers do not spell it out.
+ *
+ * Conventions shared by every call:
+ *  - Q, K, V, O are contiguous [B, H, N, D] tensors (row-major, D fastest),
+ *    in DSA_BF16 or DSA_F32.  D is 64 or 128; block is 64 or 128.
+ *  - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *    stated otherwise; the library keeps no reference after a call returns
+ *    and allocates no device memory.  Scratch memory is passed in as
+ *    `workspace` (size from dsa_workspace_size).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and never synchronises the host, except
+ *    dsa_device_status.
+ *  - Q/K/V/O pointers must be 16-byte aligned; float and int32 arrays 4-byte
+ *    aligned.
+ *  - Errors: every call returns a dsa_status and never aborts or traps.
+ *    DSA_ERR_INVALID_ARG  a null required pointer, an unsupported size
+ *                         (see each call), p outside (0, 1], bad alignment.
+ *    DSA_ERR_UNSUPPORTED  dtype/size combination not built, or a device
+ *                         that is not sm_100.
+ *    DSA_ERR_CUDA         a CUDA runtime error at launch; the text is
+ *                         available from dsa_last_error().
+ *    DSA_ERR_DEVICE       reported by dsa_device_status when a kernel saw
+ *                         malformed input (a CSR index out of range, a
+ *                         probability outside [0, 1]) or a bounded wait ran
+ *                         out; the kernel skipped the affected work.
+ *    On an error nothing is launched.  dsa_last_error() is per host thread.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,
+  DSA_ERR_UNSUPPORTED = 2,
+  DSA_ERR_CUDA = 3,
+  DSA_ERR_DEVICE = 4
+} dsa_status;
+
+typedef enum dsa_dtype { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
+
+/* Operation ids for dsa_workspace_size. */
+enum { DSA_OP_POOL_SCORE = 0, DSA_OP_SELECT_TOPP = 1 };
+
+/* Largest number of blocks per row that dsa_pool_score / dsa_select_topp
+ * accept (one warp sorts a row of up to 1024 blocks in registers). */
+#define DSA_MAX_BLOCKS 1024
+
+/*
+ * Bytes of scratch memory `op` needs for the given sizes (B, H, N, D,
+ * block as in the calls below).  Returns 0 for invalid sizes.
+ *   DSA_OP_POOL_SCORE : 2 * B*H*nB*D floats (pooled means).
+ *   DSA_OP_SELECT_TOPP: B*H*nB * 33 words (selection bitmaps and counts).
+ */
+size_t dsa_workspace_size(int op, int B, int H, int N, int D, int block);
+
+/*
+ * Pooled block scores and their row softmax (GSRS abstract: the cheap block
+ * importance estimate that Top-p selection consumes; Figure 4: reduced
+ * search evaluates only blocks inside the candidate mask).
+ *
+ *   q, k      [B, H, N, D] in dtype dt.
+ *   scale     score scale, > 0 (normally 1/sqrt(D)).
+ *   cand_row_ptr, cand_col
+ *             optional candidate CSR over the B*H*nB block rows (row r =
+ *             (b*H + h)*nB + i): cand_row_ptr [B*H*nB + 1] int32 ascending,
+ *             cand_col int32 in [0, nB).  Both NULL = full search.
+ *   probs     out, fp32 [B*H, nB, nB]: P_ij, exactly 0 outside C_i; a row
+ *             with no candidates is all 0.
+ *   workspace >= dsa_workspace_size(DSA_OP_POOL_SCORE, ...) bytes, 16-byte
+ *             aligned, contents ignored and overwritten.
+ * Limits: nB <= DSA_MAX_BLOCKS.
+ */
+dsa_status dsa_pool_score(const void* q, const void* k, dsa_dtype dt,
+                          int B, int H, int N, int D, int block, float scale,
+                          const int32_t* cand_row_ptr, const int32_t* cand_col,
+                          float* probs, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Per-row Top-p block selection (GSRS abstract: Top-p selection for
+ * adaptive sparsity; Figure 4: tighter thresholds keep fewer blocks).
+ *
+ * For each of the `rows` rows of `probs` ([rows, nB] fp32 in [0, 1]): order
+ * the candidate blocks by (probability desc, block index asc) and keep the
+ * shortest prefix whose exact sum (integer arithmetic on the fp32 values,
+ * independent of summation order) is >= p.  p >= 1 keeps every candidate;
+ * if no prefix reaches p every candidate is kept.
+ *
+ *   p          threshold in (0, 1], used as the fp32 value given.
+ *   cand_*     optional candidate CSR as in dsa_pool_score (row r of probs
+ *              uses candidates cand_col[cand_row_ptr[r] .. cand_row_ptr[r+1])).
+ *   row_ptr    out, int32 [rows + 1]: row_ptr[0] = 0, row_ptr[rows] = nnz.
+ *   col_idx    out, int32 [nnz], ascending within each row; the caller
+ *              provides capacity for rows * nB entries.
+ *   workspace  >= dsa_workspace_size(DSA_OP_SELECT_TOPP, ...) bytes with
+ *              B*H*nB = rows.
+ * Limits: nB <= DSA_MAX_BLOCKS.  The caller reads nnz from row_ptr[rows].
+ */
+dsa_status dsa_select_topp(const float* probs, int rows, int nB, float p,
+                           const int32_t* cand_row_ptr, const int32_t* cand_col,
+                           int32_t* row_ptr, int32_t* col_idx,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Exact block-sparse attention forward (GSRS abstract: exact attention over
+ * the selected blocks, computed FlashAttention-style with the exact weights
+ * as a by-product).
+ *
+ * For query t in block i of (b, h): o_t = sum_u softmax_u(scale q_t.k_u) v_u
+ * over the keys u < N of the blocks col_idx[row_ptr[r] .. row_ptr[r+1]),
+ * r = (b*H + h)*nB + i.
+ *
+ *   q, k, v   [B, H, N, D] in dt.   out: [B, H, N, D] in dt.
+ *   row_ptr, col_idx   CSR block mask over the B*H*nB rows (any column order).
+ *   lse       optional out, fp32 [B, H, N]: natural-log sum of exp(scale q.k)
+ *             over the attended keys; -inf for a row with no blocks.
+ *   blk_lse   optional out, fp32 [nnz, block]: blk_lse[s*block + t'] =
+ *             log sum over the keys of block col_idx[s] of exp(scale q.k)
+ *             for the t'-th query of the row's block (entries past a ragged
+ *             last block are not written).
+ * A row with no blocks gives O = 0.  bf16 runs on tcgen05 tensor cores with
+ * fp32 accumulation; fp32 (and block 64) runs on an exact-fp32 CUDA-core
+ * path.
+ */
+dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype dt,
+                        int B, int H, int N, int D, int block, float scale,
+                        const int32_t* row_ptr, const int32_t* col_idx,
+                        void* out, float* lse, float* blk_lse, void* stream);
+
+/*
+ * Exact softmax mass of each selected block (GSRS abstract: exact attention
+ * weights at negligible overhead; Figure 2: the recall of a block mask).
+ *
+ *   mass[s] = mean over the queries t of block i of exp(blk_lse[s, t] - lse_t)
+ * for every slot s of row r = (b*H + h)*nB + i.  Inputs are dsa_attn_fwd's
+ * lse [B, H, N] and blk_lse [nnz, block]; mass is fp32 [nnz], aligned with
+ * col_idx.  Over a row the masses sum to 1.
+ */
+dsa_status dsa_block_mass(const float* lse, const float* blk_lse,
+                          int B, int H, int N, int block, const int32_t* row_ptr,
+                          float* mass, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device-side
+ * error word.  Returns DSA_OK, DSA_ERR_DEVICE (details in dsa_last_error)
+ * or DSA_ERR_CUDA.
+ */
+dsa_status dsa_device_status(void* stream);
+
+/* Text of the last error on this host thread ("" if none). */
+const char* dsa_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,347 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Gates (on the same inputs):
+  * block probabilities P: max relative error 2e-5 (fp32 pooled scores);
+  * Top-p CSR: bit-exact against the oracle's exact selector run on the
+    GPU's own fp32 P;
+  * attention on the GPU's mask: bf16 max abs <= 2e-2 and mean abs <= 2e-3,
+    fp32 max abs <= 1e-4; lse within 2e-4 (bf16) / 1e-5 (fp32);
+  * block mass: abs <= 1e-3 (bf16) / 1e-5 (fp32).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_pool_b200 import ops, synth
+from oracle import dsa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: dict(o_max=2e-2, o_mean=2e-3, lse=2e-4, mass=1e-3, qmass=1e-4),
+       torch.float32: dict(o_max=1e-4, o_mean=1e-5, lse=1e-5, mass=1e-5, qmass=1e-5)}
+
+
+def np64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def head_csr(rp, col, h, nB):
+    """Rows of head h (rows h*nB .. h*nB+nB-1) of a global CSR, rebased."""
+    a, b = int(rp[h * nB]), int(rp[(h + 1) * nB])
+    return rp[h * nB:(h + 1) * nB + 1] - a, col[a:b], a
+
+
+def oracle_probs(q, k, block, scale, cand=None, heads=None):
+    B, H, N, D = q.shape
+    nB = ops.n_blocks(N, block)
+    out = {}
+    for bh in (range(B * H) if heads is None else heads):
+        b, h = divmod(bh, H)
+        qb = O.pool_blocks(np64(q[b, h]), block)
+        kb = O.pool_blocks(np64(k[b, h]), block)
+        c = None
+        if cand is not None:
+            rp, cc, _ = head_csr(cand[0], cand[1], bh, nB)
+            c = O.csr_rows(rp, cc)
+        out[bh] = O.block_probs(qb, kb, scale, c)
+    return out
+
+
+def check_probs(P_gpu, ref):
+    Pg = P_gpu.cpu().numpy().astype(np.float64)
+    for bh, Po in ref.items():
+        np.testing.assert_allclose(Pg[bh], Po, rtol=2e-5, atol=1e-9, err_msg=f"head {bh}")
+
+
+def check_select(P_gpu, p, rp_g, col_g, cand=None):
+    Pc = P_gpu.cpu().numpy().reshape(-1, P_gpu.shape[-1])
+    crp = ccol = None
+    if cand is not None:
+        crp, ccol = cand[0].cpu().numpy(), cand[1].cpu().numpy()
+    rp_o, col_o = O.topp_select(Pc, p, crp, ccol)
+    rp_g = rp_g.cpu().numpy()
+    np.testing.assert_array_equal(rp_g, rp_o)
+    np.testing.assert_array_equal(col_g.cpu().numpy()[:int(rp_g[-1])], col_o)
+
+
+def check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass, heads=None,
+                    rows=None, tol=None):
+    """Oracle attention on the GPU's mask for the given heads / query-block rows."""
+    B, H, N, D = q.shape
+    nB = ops.n_blocks(N, block)
+    tol = tol or TOL[q.dtype]
+    rp_c, col_c = rp.cpu().numpy().astype(np.int64), col.cpu().numpy().astype(np.int64)
+    out_c, lse_c = np64(out), lse.cpu().numpy().astype(np.float64)
+    blk_c, mass_c = blk.cpu().numpy().astype(np.float64), mass.cpu().numpy().astype(np.float64)
+    errs = []
+    for bh in (range(B * H) if heads is None else heads):
+        b, h = divmod(bh, H)
+        hrp, hcol, base = head_csr(rp_c, col_c, bh, nB)
+        Oo, lo, blo = O.sparse_attention_head(np64(q[b, h]), np64(k[b, h]), np64(v[b, h]),
+                                              block, scale, hrp, hcol, rows=rows)
+        Mo = O.block_mass(lo, blo, hrp, N, block)
+        sel_rows = range(nB) if rows is None else rows
+        for i in sel_rows:
+            a0, a1 = i * block, min(N, (i + 1) * block)
+            go, oo = out_c[b, h, a0:a1], Oo[a0:a1]
+            errs.append(np.abs(go - oo).ravel())
+            s0, s1 = int(hrp[i]), int(hrp[i + 1])
+            if s1 == s0:
+                assert np.all(go == 0), f"empty row {i} of head {bh} not zero"
+                assert np.all(np.isneginf(lse_c[b, h, a0:a1]))
+                continue
+            np.testing.assert_allclose(lse_c[b, h, a0:a1], lo[a0:a1], rtol=0, atol=tol["lse"] * max(1.0, np.abs(lo[a0:a1]).max()),
+                                       err_msg=f"lse head {bh} row {i}")
+            # per-query block weights exp(blk_lse - lse) and the block masses
+            gq = np.exp(blk_c[base + s0:base + s1, :a1 - a0] - lse_c[b, h, a0:a1][None, :])
+            oq = np.exp(blo[s0:s1, :a1 - a0] - lo[a0:a1][None, :])
+            np.testing.assert_allclose(gq, oq, rtol=0, atol=tol["qmass"], err_msg=f"blk_lse head {bh} row {i}")
+            np.testing.assert_allclose(mass_c[base + s0:base + s1], Mo[s0:s1], rtol=0, atol=tol["mass"],
+                                       err_msg=f"mass head {bh} row {i}")
+            np.testing.assert_allclose(mass_c[base + s0:base + s1].sum(), 1.0, atol=10 * tol["mass"])
+    e = np.concatenate(errs) if errs else np.zeros(1)
+    assert e.max() <= tol["o_max"], f"O max abs err {e.max():.3e}"
+    assert e.mean() <= tol["o_mean"], f"O mean abs err {e.mean():.3e}"
+    return float(e.max()), float(e.mean())
+
+
+def run_fixed_mask(q, k, v, block, rp, col, scale=None):
+    D = q.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    rpg, colg = rp.cuda(), col.cuda()
+    out, lse, blk = ops.attn_fwd(qg, kg, vg, rpg, colg, block, scale)
+    mass = ops.block_mass(lse, blk, rpg, block)
+    ops.device_status()
+    return scale, out, lse, blk, mass
+
+
+# --------------------------------------------------------------- pool/score --
+
+@pytest.mark.parametrize("B,H,N,D,block,dtype", [
+    (1, 2, 256, 64, 64, torch.float32),
+    (1, 3, 1000, 128, 128, torch.bfloat16),
+    (2, 1, 700, 64, 128, torch.bfloat16),
+    (1, 1, 130 * 64 + 5, 128, 64, torch.float32),     # nB = 131 > one score tile
+    (1, 1, 1024 * 64, 64, 64, torch.bfloat16),        # nB = 1024, the maximum
+])
+def test_pool_score_parity(B, H, N, D, block, dtype):
+    q, k, _ = synth.random_qkv(B, H, N, D, dtype, seed=11, scale=2.0)
+    scale = 1.0 / math.sqrt(D)
+    P = ops.pool_score(q.cuda(), k.cuda(), block, scale)
+    heads = None if B * H * ops.n_blocks(N, block) < 5000 else [0]
+    check_probs(P, oracle_probs(q, k, block, scale, heads=heads))
+    rows = P.sum(-1).cpu()
+    assert torch.all((rows - 1).abs() < 1e-5)
+
+
+def test_pool_score_reduced_candidates():
+    B, H, N, D, block = 1, 2, 3000, 128, 128
+    q, k, _ = synth.random_qkv(B, H, N, D, torch.bfloat16, seed=12, scale=2.0)
+    nB = ops.n_blocks(N, block)
+    rp, col = synth.random_csr(B * H * nB, nB, 0.3, seed=5)
+    rp[3:] = rp[3:]  # keep as drawn; some rows may be empty
+    P = ops.pool_score(q.cuda(), k.cuda(), block, None, cand=(rp.cuda(), col.cuda()))
+    check_probs(P, oracle_probs(q, k, block, 1 / math.sqrt(D), cand=(rp.numpy(), col.numpy())))
+    # exactly zero outside the candidates
+    mask = torch.zeros(B * H * nB, nB, dtype=torch.bool)
+    for r in range(B * H * nB):
+        mask[r, col[rp[r]:rp[r + 1]].long()] = True
+    assert torch.all(P.cpu().reshape(-1, nB)[~mask] == 0)
+
+
+def test_reduced_with_all_candidates_equals_full_bitwise():
+    B, H, N, D, block = 1, 2, 2048, 64, 128
+    q, k, _ = synth.random_qkv(B, H, N, D, torch.bfloat16, seed=13)
+    nB = ops.n_blocks(N, block)
+    rp = (torch.arange(B * H * nB + 1) * nB).int().cuda()
+    col = torch.arange(nB).repeat(B * H * nB).int().cuda()
+    qg, kg = q.cuda(), k.cuda()
+    Pf = ops.pool_score(qg, kg, block)
+    Pr = ops.pool_score(qg, kg, block, cand=(rp, col))
+    assert torch.equal(Pf, Pr)
+    a = ops.select_topp(Pf, 0.8)
+    b = ops.select_topp(Pr, 0.8, cand=(rp, col))
+    assert torch.equal(a[0], b[0])
+    n = int(a[0][-1])
+    assert torch.equal(a[1][:n], b[1][:n])
+
+
+# ------------------------------------------------------------------- select --
+
+@pytest.mark.parametrize("nB", [1, 5, 32, 33, 64, 100, 128, 200, 256, 300, 513, 929, 1024])
+@pytest.mark.parametrize("p", [0.3, 0.9, 0.99, 1.0])
+def test_select_bit_exact_random(nB, p):
+    g = torch.Generator().manual_seed(nB * 7 + int(p * 100))
+    rows = 37
+    z = torch.randn(rows, nB, generator=g) * 3.0
+    z[::4] = torch.round(z[::4])                      # exact ties
+    P = torch.softmax(z, -1).float()
+    P[5, : nB // 2] = 0.0                             # exact zeros
+    Pg = P.cuda()
+    rp, col = ops.select_topp(Pg, p)
+    ops.device_status()
+    check_select(Pg, p, rp, col)
+
+
+def test_select_adversarial_rows():
+    nB = 40
+    rows = []
+    rows.append([1.0 / nB] * nB)                                        # all tied
+    rows.append([0.0] * (nB - 1) + [1.0])                               # one-hot at the end
+    r = [0.0] * nB
+    r[3], r[17], r[30] = 0.5, 0.25, 0.25                                # sum hits p exactly
+    rows.append(r)
+    rows.append([2.0 ** -149 * (j % 3) for j in range(nB)])             # denormals only
+    rows.append([0.0] * nB)                                             # all zero
+    rows.append([(j % 5) * 2.0 ** -8 for j in range(nB)])               # many exact ties
+    P = torch.tensor(rows, dtype=torch.float32).cuda()
+    for p in (0.75, 2.0 ** -147, 0.5, 1.0, 0.9999999):
+        rp, col = ops.select_topp(P, p)
+        check_select(P, p, rp, col)
+
+
+def test_select_reduced_candidates_and_empty_rows():
+    rows, nB = 50, 300
+    g = torch.Generator().manual_seed(3)
+    P = torch.softmax(torch.randn(rows, nB, generator=g) * 2, -1).float()
+    rp, col = synth.random_csr(rows, nB, 0.2, seed=9)
+    counts = rp[1:] - rp[:-1]
+    # make two rows empty
+    keep = torch.ones(col.numel(), dtype=torch.bool)
+    for r in (4, 20):
+        keep[rp[r]:rp[r + 1]] = False
+    new_counts = counts.clone()
+    new_counts[4] = new_counts[20] = 0
+    col = col[keep]
+    rp = torch.zeros(rows + 1, dtype=torch.int32)
+    rp[1:] = torch.cumsum(new_counts, 0)
+    cand = (rp.cuda(), col.cuda())
+    for p in (0.5, 0.9, 1.0):
+        rpg, colg = ops.select_topp(P.cuda(), p, cand=cand)
+        check_select(P.cuda(), p, rpg, colg, cand=cand)
+        assert int(rpg[5] - rpg[4]) == 0 and int(rpg[21] - rpg[20]) == 0
+
+
+def test_device_flags_bad_candidates():
+    from dynamic_block_sparse_pool_b200 import DSAError
+    P = torch.full((2, 8), 0.125).cuda()
+    rp = torch.tensor([0, 2, 3], dtype=torch.int32).cuda()
+    col = torch.tensor([1, 9, 2], dtype=torch.int32).cuda()  # 9 >= nB
+    ops.select_topp(P, 0.5, cand=(rp, col))
+    with pytest.raises(DSAError, match="csr-index"):
+        ops.device_status()
+    ops.device_status()  # cleared
+
+
+# ---------------------------------------------------------------- attention --
+
+def _csr_with_empty(rows, nB, density, seed, empty=()):
+    rp, col = synth.random_csr(rows, nB, density, seed, min_per_row=1)
+    if not empty:
+        return rp, col
+    counts = (rp[1:] - rp[:-1]).clone()
+    keep = torch.ones(col.numel(), dtype=torch.bool)
+    for r in empty:
+        keep[rp[r]:rp[r + 1]] = False
+        counts[r] = 0
+    nrp = torch.zeros(rows + 1, dtype=torch.int32)
+    nrp[1:] = torch.cumsum(counts, 0)
+    return nrp, col[keep]
+
+
+@pytest.mark.parametrize("name,B,H,N,D,block,dtype,density,qscale", [
+    ("bf16_d128_ragged", 1, 2, 1000, 128, 128, torch.bfloat16, 0.5, 1.0),
+    ("bf16_d64_ragged", 2, 1, 700, 64, 128, torch.bfloat16, 0.6, 1.0),
+    ("bf16_d128_peaky", 1, 1, 1536, 128, 128, torch.bfloat16, 0.7, 3.0),
+    ("bf16_d128_long_rows", 1, 1, 128 * 40 + 7, 128, 128, torch.bfloat16, 0.8, 1.5),
+    ("bf16_block64_simt", 1, 2, 300, 64, 64, torch.bfloat16, 0.5, 1.0),
+    ("fp32_d128_block128", 1, 1, 333, 128, 128, torch.float32, 0.7, 1.0),
+    ("fp32_d64_block64", 1, 2, 256, 64, 64, torch.float32, 0.5, 2.0),
+])
+def test_attention_fixed_mask(name, B, H, N, D, block, dtype, density, qscale):
+    q, k, v = synth.random_qkv(B, H, N, D, dtype, seed=21, scale=1.0)
+    q = (q.float() * qscale).to(dtype)
+    nB = ops.n_blocks(N, block)
+    rows = B * H * nB
+    rp, col = _csr_with_empty(rows, nB, density, seed=4, empty=(1,) if rows > 2 else ())
+    scale, out, lse, blk, mass = run_fixed_mask(q, k, v, block, rp, col)
+    check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass)
+
+
+def test_attention_dense_matches_textbook_and_column_order():
+    B, H, N, D, block = 1, 2, 640, 128, 128
+    q, k, v = synth.random_qkv(B, H, N, D, torch.bfloat16, seed=22)
+    nB = ops.n_blocks(N, block)
+    rows = B * H * nB
+    rp = (torch.arange(rows + 1) * nB).int()
+    col = torch.arange(nB).repeat(rows).int()
+    scale, out, lse, blk, mass = run_fixed_mask(q, k, v, block, rp, col)
+    check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass)
+    # reversed column order inside each row: same O, lse; blk_lse permuted
+    col_r = torch.flip(col.view(rows, nB), [1]).reshape(-1).contiguous()
+    _, out2, lse2, blk2, _ = run_fixed_mask(q, k, v, block, rp, col_r)
+    assert (out2.float() - out.float()).abs().max().item() <= 2e-2
+    assert torch.allclose(lse2, lse, atol=1e-4, rtol=0)
+    b1 = blk.view(rows, nB, block)
+    b2 = torch.flip(blk2.view(rows, nB, block), [1])
+    fin = torch.isfinite(b1)
+    assert torch.allclose(b1[fin], b2[fin], atol=1e-3, rtol=0)
+
+
+# ------------------------------------------------------------ full pipeline --
+
+def pipeline_parity(w, seed, p, bandwidth=None, cand=None, heads=None, rows=None,
+                    prob_heads=None):
+    q, k, v = synth.make_qkv(w, seed, bandwidth=bandwidth)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    cand_g = None if cand is None else (cand[0].cuda(), cand[1].cuda())
+    P = ops.pool_score(qg, kg, w.block, scale, cand=cand_g)
+    rp, col = ops.select_topp(P, p, cand=cand_g)
+    out, lse, blk = ops.attn_fwd(qg, kg, vg, rp, col, w.block, scale)
+    mass = ops.block_mass(lse, blk, rp, w.block)
+    ops.device_status()
+    cand_np = None if cand is None else (cand[0].numpy(), cand[1].numpy())
+    check_probs(P, oracle_probs(q, k, w.block, scale, cand=cand_np, heads=prob_heads))
+    check_select(P, p, rp, col, cand=cand)
+    err = check_attention(q, k, v, w.block, scale, rp, col, out, lse, blk, mass,
+                          heads=heads, rows=rows)
+    nnz = int(rp[-1])
+    return rp.cpu(), col[:nnz].cpu(), err
+
+
+def test_pipeline_tiny_fp32():
+    pipeline_parity(synth.TINY, 0, 0.9)
+
+
+def test_pipeline_small_bf16():
+    pipeline_parity(synth.SMALL, 0, 0.95)
+
+
+def test_pipeline_cogvideox_sampled():
+    w = synth.COGVIDEOX
+    nB = w.n_blocks
+    pipeline_parity(w, 0, 0.9, heads=[0, 47], rows=[0, 1, 2, 70, nB - 1], prob_heads=[0, 5, 47])
+
+
+def test_pipeline_wan_sweep_and_reduced_search():
+    w = synth.WAN21
+    nB = w.n_blocks
+    rows = [0, 1, 300, nB - 1]
+    rp95, col95, _ = pipeline_parity(w, 0, 0.95, heads=[0], rows=rows, prob_heads=[0, 39])
+    # reduced search: candidates = the p=0.95 mask of seed 0, reselect at 0.7 on seed 1
+    pipeline_parity(w, 1, 0.7, cand=(rp95.int(), col95.int()), heads=[3], rows=rows,
+                    prob_heads=[3])
+
+
+def test_pipeline_hunyuan_schedule_ends():
+    w = synth.HUNYUAN
+    nB = w.n_blocks
+    sched = synth.hunyuan_schedule(10)
+    for step in (sched[0], sched[-1]):
+        _, p, bw, seed = step
+        pipeline_parity(w, seed, p, bandwidth=bw, heads=[0], rows=[0, 464, nB - 1],
+                        prob_heads=[0, 23])
