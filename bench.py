@@ -51,7 +51,7 @@ ATTN_TRAFFIC = {}
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("dsa", "reference"), default="dsa")
     ap.add_argument("--workload", default=synth.WAN21.name, choices=sorted(synth.WORKLOADS))
