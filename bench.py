@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--workload", default=synth.WAN21.name, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--p", type=float, default=0.9)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="use only this many heads of the workload (profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the p=1 reference run")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
@@ -281,6 +283,9 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads)
     B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
     nB = w.n_blocks
     rows = B * H * nB
