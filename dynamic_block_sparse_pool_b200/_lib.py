@@ -15,6 +15,7 @@ DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_DEVICE =
 DSA_F32, DSA_BF16 = 0, 1
 DSA_OP_POOL_SCORE, DSA_OP_SELECT_TOPP = 0, 1
 DSA_MAX_BLOCKS = 1024
+DSA_STATIC_MAX_ROWS = 32768
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_CUDA", 4: "DSA_ERR_DEVICE"}
@@ -27,6 +28,7 @@ SIGNATURES = {
     "dsa_select_topp": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_attn_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
     "dsa_block_mass": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "dsa_select_topp_static": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]),
     "dsa_device_status": (_i, [_vp]),
     "dsa_last_error": (ctypes.c_char_p, []),
     "dsa_version": (_i, []),

@@ -243,3 +243,18 @@ dsa_status dsa_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+namespace dsa {
+
+// For the library's other entry points: the current device's set-up
+// (architecture check, error word) and the per-thread error text.
+dsa_status api_checked_device(unsigned** err_word) {
+  DeviceInfo* d = nullptr;
+  const dsa_status st = device_info(&d);
+  if (st == DSA_OK) *err_word = d->err_word;
+  return st;
+}
+
+void api_set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
+}  // namespace dsa

@@ -170,6 +170,38 @@ dsa_status dsa_block_mass(const float* lse, const float* blk_lse,
                           int B, int H, int N, int block, const int32_t* row_ptr,
                           float* mass, void* stream);
 
+/* Largest `rows` that dsa_select_topp_static accepts. */
+#define DSA_STATIC_MAX_ROWS 32768
+
+/*
+ * dsa_select_topp without a workspace argument.  (No counterpart in the
+ * papers: this is a calling convention of this library.)
+ *
+ * For callers that cannot allocate device memory when they call in -- a
+ * host that gives a plugin only its input and output buffers, a service
+ * whose device memory all lives in its own pre-sized pool, a loop that must
+ * not call cudaMalloc or cudaFree because they can synchronise the device.
+ * Same arguments and results as dsa_select_topp, minus the workspace: the
+ * scratch (selection bitmaps and counts) is a fixed array inside the
+ * library, DSA_STATIC_MAX_ROWS * 33 words (about 4.3 MB), which every GPU
+ * that loads the library holds until the process exits.  The call allocates
+ * nothing.
+ *
+ *  - rows > DSA_STATIC_MAX_ROWS returns DSA_ERR_INVALID_ARG (use
+ *    dsa_select_topp with a workspace instead).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array.  Calls that may overlap on
+ *    the GPU (different streams, or several host threads) race on it and can
+ *    return wrong lists; order them on one stream or serialise them.  Each
+ *    call overwrites every scratch word it later reads, so nothing needs
+ *    clearing between calls.
+ */
+dsa_status dsa_select_topp_static(const float* probs, int rows, int nB, float p,
+                                  const int32_t* cand_row_ptr, const int32_t* cand_col,
+                                  int32_t* row_ptr, int32_t* col_idx, void* stream);
+
 /*
  * Synchronises `stream`, then reads and clears the library's device-side
  * error word.  Returns DSA_OK, DSA_ERR_DEVICE (details in dsa_last_error)
