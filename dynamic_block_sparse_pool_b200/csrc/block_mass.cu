@@ -7,8 +7,9 @@
 // mass[s] = mean over the queries t of block i of exp(blk_lse[s, t] - lse_t),
 // where blk_lse[s, t] is the log of the block's share of the softmax
 // denominator and lse_t the log of the whole denominator (both written by
-// the attention kernel).  One warp per CSR row keeps the row's lse values in
-// registers and reads each slot's block-size run of blk_lse once, coalesced.
+// the attention kernel).  One CTA per CSR row; each of its 8 warps keeps the
+// row's lse values in registers and reduces every 8th slot, reading that
+// slot's block-size run of blk_lse once, coalesced.
 #include "common.cuh"
 
 namespace dsa {
@@ -17,12 +18,12 @@ namespace {
 template <int BS>
 __global__ void __launch_bounds__(256)
 block_mass_kernel(const float* __restrict__ lse, const float* __restrict__ blk, int N,
-                  int nB, int rows, const int32_t* __restrict__ row_ptr,
-                  float* __restrict__ mass) {
+                  int nB, const int32_t* __restrict__ row_ptr, float* __restrict__ mass) {
   constexpr int PER = BS / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
-  if (r >= rows) return;
+  const int r = blockIdx.x;
+  const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
+  if (s1 <= s0) return;
   const int bh = r / nB, i = r - bh * nB;
   const int q0 = i * BS;
   const int qlen = min(BS, N - q0);
@@ -33,8 +34,8 @@ block_mass_kernel(const float* __restrict__ lse, const float* __restrict__ blk, 
     lv[m] = t < qlen ? lse[(size_t)bh * N + q0 + t] : 0.f;
   }
   const float inv = 1.0f / (float)qlen;
-  const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
-  for (int s = s0; s < s1; ++s) {
+  // the row's slots are spread over the CTA's 8 warps
+  for (int s = s0 + warp; s < s1; s += 8) {
     const float* b = blk + (size_t)s * BS;
     float acc = 0.f;
 #pragma unroll
@@ -55,11 +56,10 @@ cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, in
                               cudaStream_t s) {
   const int nB = ceil_div(N, block);
   const int rows = BH * nB;
-  const int grid = ceil_div(rows, 8);
   if (block == 64)
-    block_mass_kernel<64><<<grid, 256, 0, s>>>(lse, blk_lse, N, nB, rows, row_ptr, mass);
+    block_mass_kernel<64><<<rows, 256, 0, s>>>(lse, blk_lse, N, nB, row_ptr, mass);
   else
-    block_mass_kernel<128><<<grid, 256, 0, s>>>(lse, blk_lse, N, nB, rows, row_ptr, mass);
+    block_mass_kernel<128><<<rows, 256, 0, s>>>(lse, blk_lse, N, nB, row_ptr, mass);
   return cudaGetLastError();
 }
 
