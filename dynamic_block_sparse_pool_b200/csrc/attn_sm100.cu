@@ -5,33 +5,36 @@
 // GSRS (arXiv 2610.21129), abstract: exact attention over the selected
 // blocks inside a FlashAttention-style pass that also yields the exact
 // per-block attention weights.  DSV (arXiv 2502.07590), abstract: the work
-// per query block is skewed, so rows are small independent work items.
+// per query block is skewed, so every query block is its own work item.
 //
-// One CTA per pair of CSR rows (two query blocks, "tiles" 0 and 1, each with
-// its own list of key blocks).  320 threads in four roles:
-//   warps 0-3  softmax of tile 0     (thread t <-> query row t <-> TMEM lane t)
-//   warps 4-7  softmax of tile 1
+// One CTA per CSR row (one query block of 128 rows).  320 threads:
+//   warps 0-7  softmax: warp w owns the 16 query rows (TMEM lanes)
+//              32*(w%4) + 16*(w/4) .. +15; thread t of it owns two rows
+//              (t/4 and t/4 + 8 of those) and, in every 8-key chunk, keys
+//              2*(t%4) and 2*(t%4)+1 (the tcgen05.ld 16x256b layout), so the
+//              four threads of a quad share two rows and a row reduction is
+//              two quad shuffles; no warp waits for another
 //   warp  8    MMA issuer (one thread) and TMEM allocation (whole warp)
 //   warp  9    TMA loader (one thread)
-// Ten warps put three on some SM sub-partitions, whose 16K registers then
-// cap every thread at 168; the softmax keeps its 128 S values in registers
-// within that budget.
-// Tensor memory (512 columns): S_t at 256t .. 256t+127 (P_t, packed bf16
-// pairs, overwrites its first 64 columns), O_t at 256t+128 .. +D-1.
+// Tensor memory (512 columns): three S buffers at columns 0, 128, 256 (S of
+// block it in buffer it % 3; P, packed bf16 pairs, overwrites the first 64
+// columns of its buffer) and O at column 384.
+// Shared memory: Q, a 3-deep K ring and a 3-deep V ring of [128 x D] tiles.
 //
-// MMA issue order (each MMA in the same order as its operands are loaded):
-//   S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) PV1(1) S1(2) | ...
-// so the tensor cores work on one tile while the other tile's softmax runs.
-// tcgen05 MMAs issued by one thread execute in order, so S_t(j+1) reuses the
-// columns of P_t(j) only after PV_t(j) has read them, and the completion of
-// S_t(j+1) implies that of PV_t(j): when a softmax warp sees S_t(j+1) it may
-// rescale O_t in place.  K and V stream through separate two-stage rings.
+// Pipeline.  The MMA thread issues S(0), S(1), S(2), then for every block
+//   PV(it) [after P(it) is ready], S(it+3)
+// so two S tiles are computed ahead of the softmax, and the softmax warps
+// go from block to block without waiting for the tensor cores.  tcgen05 MMAs
+// from one thread execute in order: S(it+3) overwrites buffer it % 3 only
+// after PV(it) has read P(it) from it.
 //
 // Online softmax with a lazy reference: the running max m_ref moves only when
-// a block's max exceeds it by more than 8 (log2 units); otherwise P is
-// formed against the stale m_ref (values up to 2^8, exact in fp32 and
-// representable in bf16), which skips most O rescales.  The final O / l and
-// lse use the same reference, so the result is exact.
+// a block's max exceeds it by more than 8 (log2 units); otherwise P is formed
+// against the stale reference (values up to 2^8, exact in fp32 and bf16), so
+// O is rarely rescaled.  A rescale of O at block it first waits until PV(it-1)
+// has finished.  O / l and lse use the same reference, so the result is
+// exact.  P is written back with the 16x128b layout, which puts each
+// thread's packed key pairs exactly where the MMA reads row-major P.
 //
 // Each selected block's log-sum (for the exact block mass) is
 // m_ref + log2(sum of that block's P row), written per query row.
@@ -47,45 +50,73 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;        // query rows per tile (one query block)
-constexpr int BN = 128;        // keys per key block
+constexpr int BM = 128;         // query rows per CTA (one query block)
+constexpr int BN = 128;         // keys per key block
 constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
 constexpr int kMmaWarp = 8, kLoadWarp = 9;
+constexpr int kStages = 3;      // depth of the K ring and of the V ring
+constexpr int kSBufs = 3;       // S/P buffers in tensor memory
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 384;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // mbarrier slots
 enum : int {
   kBarQ = 0,
-  kBarKFull = 1,   // +stage (2)
-  kBarKEmpty = 3,  // +stage
-  kBarVFull = 5,   // +stage
-  kBarVEmpty = 7,  // +stage
-  kBarSFull = 9,   // +tile
-  kBarPFull = 11,  // +tile (128 arrivals)
-  kBarOFull = 13,  // +tile
-  kNumBars = 15
+  kBarKFull = 1,                        // + stage
+  kBarKEmpty = kBarKFull + kStages,     // + stage
+  kBarVFull = kBarKEmpty + kStages,     // + stage
+  kBarVEmpty = kBarVFull + kStages,     // + stage
+  kBarSFull = kBarVEmpty + kStages,     // + S buffer
+  kBarPFull = kBarSFull + kSBufs,       // + S buffer (256 arrivals)
+  kBarPVDone = kBarPFull + kSBufs,      // + (block & 1)
+  kBarOFull = kBarPVDone + 2,
+  kNumBars = kBarOFull + 1
 };
 
 template <int D>
 struct SmemLayout {
-  static constexpr int kTile = BM * D * 2;  // bytes of one [128 x D] bf16 tile
-  static constexpr int kSub = BM * 64 * 2;  // one 128B-swizzled [128 x 64] sub-tile
-  static constexpr int kQ = 0;              // Q of tiles 0, 1
-  static constexpr int kK = 2 * kTile;      // K ring, 2 stages
-  static constexpr int kV = 4 * kTile;      // V ring, 2 stages
-  static constexpr int kBar = 6 * kTile;
-  static constexpr int kSlot = kBar + 8 * kNumBars;  // TMEM base, abort flag
+  static constexpr int kTile = BM * D * 2;                // one [128 x D] bf16 tile
+  static constexpr int kSub = BM * 64 * 2;                // one 128B-swizzled [128 x 64] sub-tile
+  static constexpr int kQ = 0;
+  static constexpr int kK = kTile;                        // K ring
+  static constexpr int kV = kK + kStages * kTile;         // V ring
+  static constexpr int kBar = kV + kStages * kTile;
+  static constexpr int kRagged = kBar + 8 * kNumBars;     // uint32 [32]: list positions of the ragged block
+  static constexpr int kSlot = kRagged + 32 * 4;          // TMEM base, abort flag
   static constexpr int kBytes = kSlot + 16;
-  static constexpr int kAlloc = kBytes + 1024;       // room to align tiles to 1024 B
-};
-
-struct Tile {
-  int bh, q0, qlen, s0, n;
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// 2^x on the multi-function unit (the PTX approximate base-2 exponential).
+__device__ __forceinline__ float exp2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe, for x <= 8 (softmax arguments here never exceed the
+// rescale threshold).  Cody-Waite style reduction x = n + f with n = round(x)
+// (the 1.5 * 2^23 rounding constant) and |f| <= 1/2, then a degree-4
+// polynomial for 2^f fitted for minimum maximum relative error on
+// [-1/2, 1/2] (Lawson's iteratively reweighted least squares; max relative
+// error 2.7e-6 when evaluated in fp32), then n is added to the exponent
+// field.  Arguments below -125 (including -inf) give 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.0f);
+  const float t = xc + 12582912.0f;
+  const float f = xc - (t - 12582912.0f);
+  float p = fmaf(0x1.3997d4p-7f, f, 0x1.ca1442p-5f);
+  p = fmaf(p, f, 0x1.ec06dap-3f);
+  p = fmaf(p, f, 0x1.62e0dcp-1f);
+  p = fmaf(p, f, 0x1.ffffe8p-1f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  const float y = __int_as_float(__float_as_int(p) + (n << 23));
+  return x < -125.0f ? 0.0f : y;
+}
 
 template <int D>
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row, int bh,
@@ -99,7 +130,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, int N, int nB, int rows,
+                      const __grid_constant__ CUtensorMap tmV, int N, int nB,
                       float scale_log2, const int32_t* __restrict__ row_ptr,
                       const int32_t* __restrict__ col_idx, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ lse, float* __restrict__ blk_lse, unsigned* err) {
@@ -107,56 +138,33 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, true);
   constexpr uint32_t kTileBytes = L::kTile;
+  constexpr int kHalfD = D / 2;   // O columns owned by each half of a row
 
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t base = smem_u32(smem);
+  if (base & 1023u) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) flag_error(err, kErrAlign);
+    return;
+  }
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV;
   const uint32_t bars = base + L::kBar;
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kSlot);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kSlot + 4);
+  uint32_t* ragged_bits = reinterpret_cast<uint32_t*>(smem + L::kRagged);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlot + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = blockIdx.x;
+  const int bh = r / nB, qi = r - bh * nB;
+  const int q0 = qi * BM;
+  const int qlen = min(BM, N - q0);
+  const int kv_last = N - (nB - 1) * BN;  // keys in the last (possibly ragged) block
 
-  // ---- the two rows of this CTA --------------------------------------------
-  Tile tl[2];
-  bool bad[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int r = 2 * blockIdx.x + t;
-    tl[t].bh = 0; tl[t].q0 = 0; tl[t].qlen = 0; tl[t].s0 = 0; tl[t].n = 0;
-    bad[t] = false;
-    if (r < rows) {
-      const int bh = r / nB, i = r - bh * nB;
-      tl[t].bh = bh;
-      tl[t].q0 = i * BM;
-      tl[t].qlen = min(BM, N - i * BM);
-      const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
-      tl[t].s0 = s0;
-      tl[t].n = s1 - s0;
-      bad[t] = s0 < 0 || s1 < s0;
-      if (!bad[t])
-        for (int e = s0 + tid; e < s1; e += kThreads) {
-          const int j = col_idx[e];
-          bad[t] |= (j < 0 || j >= nB);
-        }
-    }
-  }
-
+  if (tid < 32) ragged_bits[tid] = 0u;
   if (warp == kMmaWarp) {
     if (lane == 0) {
-      mbar_init(bar(kBarQ), 1);
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(bar(kBarKFull + s), 1);
-        mbar_init(bar(kBarKEmpty + s), 1);
-        mbar_init(bar(kBarVFull + s), 1);
-        mbar_init(bar(kBarVEmpty + s), 1);
-        mbar_init(bar(kBarSFull + s), 1);
-        mbar_init(bar(kBarPFull + s), 128);
-        mbar_init(bar(kBarOFull + s), 1);
-      }
+      for (int i = 0; i < kNumBars; ++i)
+        mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kSBufs) ? kSoftmaxThreads : 1);
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -169,121 +177,106 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
+  __syncthreads();
+
+  // validate the row and mark where the ragged last key block sits in it
+  int s0 = row_ptr[r], s1 = row_ptr[r + 1];
+  bool bad = s0 < 0 || s1 < s0;
+  if (!bad)
+    for (int e = s0 + tid; e < s1; e += kThreads) {
+      const int j = col_idx[e];
+      bad |= (j < 0 || j >= nB);
+      if (j == nB - 1 && kv_last < BN && e - s0 < 1024)
+        atomicOr(&ragged_bits[(e - s0) >> 5], 1u << ((e - s0) & 31));
+    }
   tc_fence_before();
-  const bool bad0 = __syncthreads_or(bad[0]);
-  const bool bad1 = __syncthreads_or(bad[1]);
+  const bool any_bad = __syncthreads_or(bad);
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (bad0) {
+  if (any_bad) {
     if (tid == 0) flag_error(err, kErrCsrIndex | kErrRowPtr);
-    tl[0].n = 0;
+    s1 = s0;
   }
-  if (bad1) {
-    if (tid == 0) flag_error(err, kErrCsrIndex | kErrRowPtr);
-    tl[1].n = 0;
-  }
-  const int n0 = tl[0].n, n1 = tl[1].n;
-  const int nmax = n0 > n1 ? n0 : n1;
+  const int n = s1 - s0;
 
   if (warp == kLoadWarp) {
     // ---------------------------------------------------------------- loader
-    if (lane == 0 && nmax > 0) {
+    if (lane == 0 && n > 0) {
+      // K runs kKLead blocks ahead of V: S(it) needs K(it) a block earlier
+      // than PV(it) needs V(it), and K(it + 3)'s slot frees as soon as S(it)
+      // is done, so K gets about three block periods to arrive from L2.
+      constexpr int kKLead = 2;
       bool ok = true;
-      uint32_t kc = 0, vc = 0;           // loads issued into each ring
-      uint32_t k_used = 0, v_used = 0;   // bit s: stage s has received a load
-      uint32_t k_last_ph = 0, v_last_ph = 0;  // bit s: parity of its last load
-      mbar_expect_tx(bar(kBarQ), (n0 > 0 ? kTileBytes : 0) + (n1 > 0 ? kTileBytes : 0));
-      if (n0 > 0) tma_tile<D>(sQ, &tmQ, tl[0].q0, tl[0].bh, bar(kBarQ));
-      if (n1 > 0) tma_tile<D>(sQ + kTileBytes, &tmQ, tl[1].q0, tl[1].bh, bar(kBarQ));
-      auto load_k = [&](int t, int it) {
-        const uint32_t s = kc & 1u, ph = ((kc >> 1) & 1u) ^ 1u;
-        if (!(ok = ok && mbar_wait(bar(kBarKEmpty + s), ph))) return;
-        const int j = col_idx[tl[t].s0 + it];
-        mbar_expect_tx(bar(kBarKFull + s), kTileBytes);
-        tma_tile<D>(sK + s * kTileBytes, &tmK, j * BN, tl[t].bh, bar(kBarKFull + s));
-        k_used |= 1u << s;
-        k_last_ph = (k_last_ph & ~(1u << s)) | (((kc >> 1) & 1u) << s);
-        ++kc;
-      };
-      auto load_v = [&](int t, int it) {
-        const uint32_t s = vc & 1u, ph = ((vc >> 1) & 1u) ^ 1u;
-        if (!(ok = ok && mbar_wait(bar(kBarVEmpty + s), ph))) return;
-        const int j = col_idx[tl[t].s0 + it];
-        mbar_expect_tx(bar(kBarVFull + s), kTileBytes);
-        tma_tile<D>(sV + s * kTileBytes, &tmV, j * BN, tl[t].bh, bar(kBarVFull + s));
-        v_used |= 1u << s;
-        v_last_ph = (v_last_ph & ~(1u << s)) | (((vc >> 1) & 1u) << s);
-        ++vc;
-      };
-      if (n0 > 0) load_k(0, 0);
-      if (n1 > 0 && ok) load_k(1, 0);
-      for (int it = 0; it < nmax && ok && !*abort_flag; ++it) {
-        if (it < n0) {
-          load_v(0, it);
-          if (it + 1 < n0 && ok) load_k(0, it + 1);
+      int k_issued = 0, v_issued = 0;  // blocks whose K / V loads were issued
+      mbar_expect_tx(bar(kBarQ), kTileBytes);
+      tma_tile<D>(sQ, &tmQ, q0, bh, bar(kBarQ));
+      for (int step = 0; step < n + kKLead && ok; ++step) {
+        if (step < n) {
+          const int it = step, s = it % kStages;
+          const int j = col_idx[s0 + it];
+          ok = mbar_wait(bar(kBarKEmpty + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
+          if (!ok) break;
+          mbar_expect_tx(bar(kBarKFull + s), kTileBytes);
+          tma_tile<D>(sK + s * kTileBytes, &tmK, j * BN, bh, bar(kBarKFull + s));
+          k_issued = it + 1;
         }
-        if (it < n1 && ok) {
-          load_v(1, it);
-          if (it + 1 < n1 && ok) load_k(1, it + 1);
+        if (step >= kKLead) {
+          const int it = step - kKLead, s = it % kStages;
+          const int j = col_idx[s0 + it];
+          ok = mbar_wait(bar(kBarVEmpty + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
+          if (!ok) break;
+          mbar_expect_tx(bar(kBarVFull + s), kTileBytes);
+          tma_tile<D>(sV + s * kTileBytes, &tmV, j * BN, bh, bar(kBarVFull + s));
+          v_issued = it + 1;
         }
       }
-      if (!ok || *abort_flag) {
+      if (!ok) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
         // let the loads still in flight land before shared memory is released
-        for (int s = 0; s < 2; ++s) {
-          if ((k_used >> s) & 1u) mbar_wait(bar(kBarKFull + s), (k_last_ph >> s) & 1u);
-          if ((v_used >> s) & 1u) mbar_wait(bar(kBarVFull + s), (v_last_ph >> s) & 1u);
-        }
-        mbar_wait(bar(kBarQ), 0);
+        for (int b = k_issued - kStages > 0 ? k_issued - kStages : 0; b < k_issued; ++b)
+          mbar_wait(bar(kBarKFull + b % kStages), (uint32_t)(b / kStages) & 1u);
+        for (int b = v_issued - kStages > 0 ? v_issued - kStages : 0; b < v_issued; ++b)
+          mbar_wait(bar(kBarVFull + b % kStages), (uint32_t)(b / kStages) & 1u);
+        mbar_wait(bar(kBarQ), 0u);
       }
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issuer
-    if (lane == 0 && nmax > 0) {
-      bool ok = mbar_wait(bar(kBarQ), 0);
-      uint32_t kc = 0, vc = 0;
-      auto issue_s = [&](int t) {
-        const uint32_t s = kc & 1u, ph = (kc >> 1) & 1u;
-        if (!(ok = ok && mbar_wait(bar(kBarKFull + s), ph))) return;
+    if (lane == 0 && n > 0) {
+      bool ok = mbar_wait(bar(kBarQ), 0u);
+      auto issue_s = [&](int it) {
+        const int s = it % kStages;
+        if (!(ok = ok && mbar_wait(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u))) return;
         tc_fence_after();
-        const uint32_t q = sQ + t * kTileBytes, k = sK + s * kTileBytes;
+        const uint32_t k = sK + s * kTileBytes;
+        const uint32_t d = tmem + 128u * (uint32_t)(it % kSBufs);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
-          mma_ss(tmem + 256u * t, smem_desc_sw128(q + off, 16, 1024),
-                 smem_desc_sw128(k + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(k + off, 16, 1024),
+                 kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBarKEmpty + s));
-        mma_commit(bar(kBarSFull + t));
-        ++kc;
+        mma_commit(bar(kBarSFull + it % kSBufs));
       };
-      auto issue_pv = [&](int t, int it, int n) {
-        if (!(ok = ok && mbar_wait(bar(kBarPFull + t), (uint32_t)it & 1u))) return;
-        const uint32_t s = vc & 1u, ph = (vc >> 1) & 1u;
-        if (!(ok = ok && mbar_wait(bar(kBarVFull + s), ph))) return;
+      for (int it = 0; it < n && it < kSBufs; ++it) issue_s(it);
+      for (int it = 0; it < n && ok && !*abort_flag; ++it) {
+        const int b = it % kSBufs, s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kSBufs) & 1u;
+        if (!(ok = mbar_wait(bar(kBarPFull + b), ph))) break;
+        if (!(ok = mbar_wait(bar(kBarVFull + s), (uint32_t)(it / kStages) & 1u))) break;
         tc_fence_after();
         const uint32_t v = sV + s * kTileBytes;
+        const uint32_t p = tmem + 128u * (uint32_t)b;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
-                 smem_desc_sw128(v + kk * 2048, L::kSub, 1024), kIdescO,
+          mma_ts(tmem + kTmemO, p + kk * 8, smem_desc_sw128(v + kk * 2048, L::kSub, 1024), kIdescO,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(kBarVEmpty + s));
-        if (it == n - 1) mma_commit(bar(kBarOFull + t));
-        ++vc;
-      };
-      if (n0 > 0 && ok) issue_s(0);
-      if (n1 > 0 && ok) issue_s(1);
-      for (int it = 0; it < nmax && ok && !*abort_flag; ++it) {
-        if (it < n0) {
-          issue_pv(0, it, n0);
-          if (it + 1 < n0 && ok) issue_s(0);
-        }
-        if (it < n1 && ok) {
-          issue_pv(1, it, n1);
-          if (it + 1 < n1 && ok) issue_s(1);
-        }
+        mma_commit(bar(kBarPVDone + (it & 1)));
+        if (it == n - 1) mma_commit(bar(kBarOFull));
+        if (it + kSBufs < n) issue_s(it + kSBufs);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -292,114 +285,179 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int t = warp >> 2;
-    const Tile T = t ? tl[1] : tl[0];
-    const int row = tid - 128 * t;
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + 256u * t + lane_off;
-    const uint32_t tO = tS + 128u;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int it = 0; it < T.n; ++it) {
-      ok = warp_all(mbar_wait(bar(kBarSFull + t), (uint32_t)it & 1u)) && !warp_all(*abort_flag != 0);
-      if (!ok) break;
+    const int rbase = 32 * (warp & 3) + 16 * (warp >> 2);  // first of the warp's 16 rows
+    const int t0 = lane & 3;
+    const int ra = rbase + (lane >> 2), rb = ra + 8;         // this thread's two rows
+    const uint32_t lane_off = (uint32_t)rbase << 16;
+    float mref_a = -INFINITY, mref_b = -INFINITY;  // reference maxima (log2 units)
+    float l_a = 0.f, l_b = 0.f;                    // this thread's share of the row sums
+    bool failed = false;
+    for (int it = 0; it < n; ++it) {
+      const int b = it % kSBufs;
+      const uint32_t tS = tmem + lane_off + 128u * (uint32_t)b;
+      if (!warp_all(mbar_wait(bar(kBarSFull + b), (uint32_t)(it / kSBufs) & 1u)) ||
+          warp_all(*abort_flag != 0)) {
+        failed = true;
+        break;
+      }
       tc_fence_after();
-      const int j = col_idx[T.s0 + it];
-      uint32_t sv[128];
+      // sv[4k + u]: row ra, key 8k + 2*t0 + u; sv[4k + 2 + u]: row rb, same key
+      uint32_t sv[64];
+      tmem_ld16x256b_x16(tS, sv);
+      tmem_wait_ld_regs64(sv);
+      const bool rag = it < 1024 ? ((ragged_bits[it >> 5] >> (it & 31)) & 1u)
+                                 : (kv_last < BN && col_idx[s0 + it] == nB - 1);
+      if (rag) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
+        for (int k = 0; k < 16; ++k)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_wait_ld_regs(*reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
-      const int kv_len = min(BN, N - j * BN);
-      if (kv_len < BN) {
-#pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (e >= kv_len) sv[e] = __float_as_uint(-INFINITY);
+          for (int u = 0; u < 2; ++u)
+            if (8 * k + 2 * t0 + u >= kv_last) {
+              sv[4 * k + u] = __float_as_uint(-INFINITY);
+              sv[4 * k + 2 + u] = __float_as_uint(-INFINITY);
+            }
       }
-      float mx = __uint_as_float(sv[0]);
+      float ma4[4], mb4[4];
 #pragma unroll
-      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
-      const float mb = mx * scale_log2;
-      const bool need = mb > m_ref + kRescaleThreshold;
-      const bool warp_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.0f;
-      if (need) {
-        alpha = exp2f(m_ref - mb);  // 0 on the first block
-        l *= alpha;
-        m_ref = mb;
+      for (int u = 0; u < 4; ++u) {
+        ma4[u] = fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1]));
+        mb4[u] = fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]));
       }
-      float rs = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(fmaf(__uint_as_float(sv[32 * c + 2 * e]), scale_log2, -m_ref));
-          const float p1 = exp2f(fmaf(__uint_as_float(sv[32 * c + 2 * e + 1]), scale_log2, -m_ref));
-          rs += p0 + p1;
-          const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // .x = p0, low half
-          pk[e] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        tmem_st16(tS + c * 16, pk);
+      for (int k = 4; k < 16; ++k) {
+        ma4[k & 3] = fmaxf(ma4[k & 3], fmaxf(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1])));
+        mb4[k & 3] = fmaxf(mb4[k & 3], fmaxf(__uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3])));
       }
-      // O_t holds the sum up to block it-1 (its PV completed before S_t(it));
-      // move it to the new reference before PV_t(it) accumulates onto it
+      float ma = fmaxf(fmaxf(ma4[0], ma4[1]), fmaxf(ma4[2], ma4[3]));
+      float mb = fmaxf(fmaxf(mb4[0], mb4[1]), fmaxf(mb4[2], mb4[3]));
+      ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+      ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+      const float xa = ma * scale_log2, xb = mb * scale_log2;
+      const bool need_a = xa > mref_a + kRescaleThreshold;
+      const bool need_b = xb > mref_b + kRescaleThreshold;
+      const bool warp_need = __any_sync(0xffffffffu, need_a || need_b);
+      float alpha_a = 1.0f, alpha_b = 1.0f;
+      if (need_a) {
+        alpha_a = exp2f(mref_a - xa);  // 0 on the first block
+        l_a *= alpha_a;
+        mref_a = xa;
+      }
+      if (need_b) {
+        alpha_b = exp2f(mref_b - xb);
+        l_b *= alpha_b;
+        mref_b = xb;
+      }
+      // P = 2^(S*scale*log2e - m_ref); pk[2k]: row ra, packed keys (8k+2t0, 8k+2t0+1),
+      // pk[2k+1]: row rb -- the 16x128b layout of packed column 4k + t0
+      float rsa[2] = {0.f, 0.f}, rsb[2] = {0.f, 0.f};
+      uint32_t pk[32];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float a0 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k]), scale_log2, -mref_a));
+        const float a1 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k + 1]), scale_log2, -mref_a));
+        const float b0 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k + 2]), scale_log2, -mref_b));
+        const float b1 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k + 3]), scale_log2, -mref_b));
+        rsa[k & 1] += a0 + a1;
+        rsb[k & 1] += b0 + b1;
+        const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1);  // .x = lower key, low half
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(b0, b1);
+        pk[2 * k] = *reinterpret_cast<const uint32_t*>(&ha);
+        pk[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&hb);
+      }
+      tmem_st16x128b_x16(tS, pk);
+      const float rs_a = rsa[0] + rsa[1], rs_b = rsb[0] + rsb[1];
       if (warp_need && it > 0) {
+        // O holds the sum through block it-1; wait for PV(it-1), then move O to
+        // the new reference before PV(it) accumulates onto it
+        const int pb = (it - 1) & 1;
+        if (!warp_all(mbar_wait(bar(kBarPVDone + pb), (uint32_t)((it - 1) >> 1) & 1u))) {
+          *abort_flag = 1;
+        } else {
+          tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld_regs(o);
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_off + kTmemO + 64 * c;
+            tmem_ld16x256b_x8(ta, o);
+            tmem_wait_ld_regs(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + c * 32, o);
+            for (int k = 0; k < 8; ++k) {
+              o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * alpha_a);
+              o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * alpha_a);
+              o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * alpha_b);
+              o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * alpha_b);
+            }
+            tmem_st16x256b_x8(ta, o);
+          }
         }
       }
-      l += rs;
+      l_a += rs_a;
+      l_b += rs_b;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + t));
-      if (blk_lse != nullptr && row < T.qlen)
-        blk_lse[(size_t)(T.s0 + it) * BN + row] = (m_ref + log2f(rs)) * kLn2;
+      mbar_arrive(bar(kBarPFull + b));
+      if (blk_lse != nullptr) {
+        // the block's share of each row's denominator: sum over the quad
+        float ta = rs_a + __shfl_xor_sync(0xffffffffu, rs_a, 1);
+        float tb = rs_b + __shfl_xor_sync(0xffffffffu, rs_b, 1);
+        ta += __shfl_xor_sync(0xffffffffu, ta, 2);
+        tb += __shfl_xor_sync(0xffffffffu, tb, 2);
+        if (t0 == 0) {
+          if (ra < qlen) blk_lse[(size_t)(s0 + it) * BN + ra] = (mref_a + log2f(ta)) * kLn2;
+          if (rb < qlen) blk_lse[(size_t)(s0 + it) * BN + rb] = (mref_b + log2f(tb)) * kLn2;
+        }
+      }
     }
-    if (!ok) {
+
+    if (failed) {
       *abort_flag = 1;
       flag_error(err, kErrTimeout);
-    } else if (T.n > 0) {
-      ok = warp_all(mbar_wait(bar(kBarOFull + t), 0u));
-      if (!ok) {
+    } else if (n > 0) {
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      if (!warp_all(mbar_wait(bar(kBarOFull), 0u))) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
       } else {
         tc_fence_after();
-        __nv_bfloat16* orow = out + ((size_t)T.bh * N + T.q0 + row) * D;
-        const float inv_l = 1.0f / l;
+        const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
+        __nv_bfloat16* oa = out + ((size_t)bh * N + q0 + ra) * D + 2 * t0;
+        __nv_bfloat16* ob = out + ((size_t)bh * N + q0 + rb) * D + 2 * t0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
+          tmem_ld16x256b_x8(tmem + lane_off + kTmemO + 64 * c, o);
           tmem_wait_ld_regs(o);
-          if (row < T.qlen) {
-            uint4 pkt[4];
-            uint32_t* w = reinterpret_cast<uint32_t*>(pkt);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv_l,
-                                                             __uint_as_float(o[2 * e + 1]) * inv_l);
-              w[e] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) dst[u] = pkt[u];
+          for (int k = 0; k < 8; ++k) {
+            const __nv_bfloat162 ha = __floats2bfloat162_rn(__uint_as_float(o[4 * k]) * inv_a,
+                                                            __uint_as_float(o[4 * k + 1]) * inv_a);
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[4 * k + 2]) * inv_b,
+                                                            __uint_as_float(o[4 * k + 3]) * inv_b);
+            if (ra < qlen) *reinterpret_cast<__nv_bfloat162*>(oa + 64 * c + 8 * k) = ha;
+            if (rb < qlen) *reinterpret_cast<__nv_bfloat162*>(ob + 64 * c + 8 * k) = hb;
           }
         }
-        if (lse != nullptr && row < T.qlen) lse[(size_t)T.bh * N + T.q0 + row] = (m_ref + log2f(l)) * kLn2;
+        if (t0 == 0 && lse != nullptr) {
+          if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
+          if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
+        }
       }
-    } else if (row < T.qlen) {
-      uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)T.bh * N + T.q0 + row) * D);
+    } else {
+      const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (lse != nullptr) lse[(size_t)T.bh * N + T.q0 + row] = -INFINITY;
+      for (int k = 0; k < D / 8; ++k) {
+        if (ra < qlen) *reinterpret_cast<__nv_bfloat162*>(out + ((size_t)bh * N + q0 + ra) * D + 8 * k + 2 * t0) = z;
+        if (rb < qlen) *reinterpret_cast<__nv_bfloat162*>(out + ((size_t)bh * N + q0 + rb) * D + 8 * k + 2 * t0) = z;
+      }
+      if (t0 == 0 && lse != nullptr) {
+        if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = -INFINITY;
+        if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = -INFINITY;
+      }
     }
   }
 
@@ -449,14 +507,14 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                      void* out, float* lse, float* blk_lse, unsigned* err, cudaStream_t s) {
   const int nB = ceil_div(N, BN);
   const int rows = BH * nB;
-  const int smem = SmemLayout<D>::kAlloc;
+  const int smem = SmemLayout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
-  attn_fwd_sm100_kernel<D><<<ceil_div(rows, 2), kThreads, smem, s>>>(
-      mq, mk, mv, N, nB, rows, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out),
-      lse, blk_lse, err);
+  attn_fwd_sm100_kernel<D><<<rows, kThreads, smem, s>>>(
+      mq, mk, mv, N, nB, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out), lse,
+      blk_lse, err);
   return cudaGetLastError();
 }
 

@@ -13,6 +13,7 @@ enum : unsigned {
   kErrRowPtr = 2u,       // a row_ptr entry that is negative or decreasing
   kErrProb = 4u,         // a probability outside [0, 1] or NaN
   kErrTimeout = 8u,      // a bounded wait on an mbarrier ran out
+  kErrAlign = 16u,       // dynamic shared memory not 1024-byte aligned
 };
 
 // Upper bound for one mbarrier wait before a kernel gives up (nanoseconds).
