@@ -244,21 +244,52 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
+      // Every shared-memory descriptor is formed once here: the issuing
+      // thread shares its SM sub-partition with two busy softmax warps, so
+      // each MMA should cost it as few instructions as possible.
+      uint64_t dq[D / 16], dk[kStages][D / 16], dv[kStages][BN / 16];
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
+        dq[kk] = smem_desc_sw128(sQ + off, 16, 1024);
+#pragma unroll
+        for (int st = 0; st < kStages; ++st)
+          dk[st][kk] = smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024);
+      }
+#pragma unroll
+      for (int st = 0; st < kStages; ++st)
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          dv[st][kk] = smem_desc_sw128(sV + st * kTileBytes + kk * 2048, L::kSub, 1024);
       bool ok = mbar_wait(bar(kBarQ), 0u);
+      // S(it) = Q K^T into buffer it % 3; the ring stage is dispatched to
+      // compile-time indices so the descriptors stay in registers
+      auto s_mmas = [&](uint32_t d, const uint64_t (&k)[D / 16]) {
+        mma_ss(d, dq[0], k[0], kIdescS, 0u);
+#pragma unroll
+        for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, dq[kk], k[kk], kIdescS);
+      };
       auto issue_s = [&](int it) {
         const int s = it % kStages;
         if (!(ok = ok && mbar_wait(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u))) return;
         tc_fence_after();
-        const uint32_t k = sK + s * kTileBytes;
         const uint32_t d = tmem + 128u * (uint32_t)(it % kSBufs);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
-          mma_ss(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(k + off, 16, 1024),
-                 kIdescS, kk > 0 ? 1u : 0u);
+        switch (s) {
+          case 0: s_mmas(d, dk[0]); break;
+          case 1: s_mmas(d, dk[1]); break;
+          default: s_mmas(d, dk[2]); break;
         }
         mma_commit(bar(kBarKEmpty + s));
         mma_commit(bar(kBarSFull + it % kSBufs));
+      };
+      // O += P(it) V(it), P from tensor memory
+      auto pv_mmas = [&](uint32_t p, bool first, const uint64_t (&v)[BN / 16]) {
+        if (first)
+          mma_ts(tmem + kTmemO, p, v[0], kIdescO, 0u);
+        else
+          mma_ts_acc(tmem + kTmemO, p, v[0], kIdescO);
+#pragma unroll
+        for (int kk = 1; kk < BN / 16; ++kk) mma_ts_acc(tmem + kTmemO, p + kk * 8, v[kk], kIdescO);
       };
       for (int it = 0; it < n && it < kSBufs; ++it) issue_s(it);
       for (int it = 0; it < n && ok && !*abort_flag; ++it) {
@@ -267,12 +298,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (!(ok = mbar_wait(bar(kBarPFull + b), ph))) break;
         if (!(ok = mbar_wait(bar(kBarVFull + s), (uint32_t)(it / kStages) & 1u))) break;
         tc_fence_after();
-        const uint32_t v = sV + s * kTileBytes;
         const uint32_t p = tmem + 128u * (uint32_t)b;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + kTmemO, p + kk * 8, smem_desc_sw128(v + kk * 2048, L::kSub, 1024), kIdescO,
-                 (it > 0 || kk > 0) ? 1u : 0u);
+        switch (s) {
+          case 0: pv_mmas(p, it == 0, dv[0]); break;
+          case 1: pv_mmas(p, it == 0, dv[1]); break;
+          default: pv_mmas(p, it == 0, dv[2]); break;
+        }
         mma_commit(bar(kBarVEmpty + s));
         mma_commit(bar(kBarPVDone + (it & 1)));
         if (it == n - 1) mma_commit(bar(kBarOFull));
