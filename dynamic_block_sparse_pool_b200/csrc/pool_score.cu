@@ -9,9 +9,9 @@
 // Kernel 1 (pool_means): one CTA per (block, head, Q-or-K); 16-byte loads,
 //   fp32 accumulation, mean over the block's actual rows.  HBM-bound: reads
 //   Q and K once.
-// Kernel 2 (block_scores): one CTA per (32 query-block rows, head).  The 32
-//   pooled queries stay in shared memory; pooled keys stream through in
-//   tiles of 64; the 32 x nB raw scores stay in shared memory for the row
+// Kernel 2 (block_scores): one CTA per (32 query-block rows, head): a
+//   register-tiled fp32 product of the 32 pooled queries with tiles of 64
+//   pooled keys; the 32 x nB raw scores stay in shared memory for the row
 //   softmax, which writes P once, coalesced.
 #include "common.cuh"
 
@@ -59,16 +59,22 @@ pool_means_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int n
 
 constexpr int kRows = 32;   // query-block rows per CTA
 constexpr int kCols = 64;   // key blocks per score tile
+constexpr int kDc = 32;     // head-dim slice staged in shared memory at a time
 
 __host__ __device__ constexpr int scores_pad(int nB) { return ceil_div(nB, kCols) * kCols; }
 
-template <int D>
 __host__ __device__ constexpr size_t scores_smem_bytes(int nB) {
-  return sizeof(float) * ((size_t)kRows * (D + 1) + (size_t)kCols * (D + 1) +
+  return sizeof(float) * ((size_t)kDc * (kRows + 1) + (size_t)kDc * (kCols + 1) +
                           (size_t)kRows * scores_pad(nB)) +
          sizeof(uint32_t) * kRows * 32;
 }
 
+// Scores of 32 pooled queries against all pooled keys of a head, then the row
+// softmax.  The 32 x 64 score tile is a register-tiled fp32 product: thread
+// (ty, tx) of a 16 x 16 grid computes rows 2*ty, 2*ty+1 and columns
+// tx + 16*c (c < 4): 6 shared-memory loads per 8 FMAs, from transposed
+// slices of 32 head dimensions padded to odd strides (conflict-free both when
+// staged and when read).
 template <int D>
 __global__ void __launch_bounds__(256)
 block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
@@ -76,9 +82,10 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
                     const int32_t* __restrict__ cand_col, float* __restrict__ probs,
                     unsigned* err) {
   extern __shared__ float sm[];
-  float* qs = sm;                                  // [kRows][D+1]
-  float* ks = qs + kRows * (D + 1);                // [kCols][D+1]
-  float* sc = ks + kCols * (D + 1);                // [kRows][pad]
+  constexpr int QS = kRows + 1, KS = kCols + 1;    // padded strides
+  float* qs = sm;                                  // [kDc][QS]   (transposed)
+  float* ks = qs + kDc * QS;                       // [kDc][KS]   (transposed)
+  float* sc = ks + kDc * KS;                       // [kRows][pad]
   const int pad = scores_pad(nB);
   uint32_t* cbits = reinterpret_cast<uint32_t*>(sc + kRows * pad);  // [kRows][32]
 
@@ -88,10 +95,6 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
   const int nrows = min(kRows, nB - i0);
   const bool reduced = cand_row_ptr != nullptr;
 
-  for (int idx = tid; idx < kRows * D; idx += 256) {
-    const int rr = idx / D, d = idx - rr * D;
-    qs[rr * (D + 1) + d] = rr < nrows ? qbar[((size_t)bh * nB + i0 + rr) * D + d] : 0.f;
-  }
   if (reduced) {
     for (int idx = tid; idx < kRows * 32; idx += 256) cbits[idx] = 0u;
     __syncthreads();
@@ -114,8 +117,8 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
   }
   __syncthreads();
 
-  const int rr = tid >> 3;   // score row of this thread
-  const int c0 = tid & 7;    // first of its 8 columns (stride 8)
+  const int ty = tid >> 4, tx = tid & 15;
+  const float* qhead = qbar + ((size_t)bh * nB + i0) * D;
   for (int t0 = 0; t0 < nB; t0 += kCols) {
     if (reduced) {
       // skip a tile that holds no candidate of any of this CTA's rows
@@ -126,25 +129,42 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
       }
       if (!__syncthreads_or(any)) continue;
     }
-    for (int idx = tid; idx < kCols * D; idx += 256) {
-      const int cc = idx / D, d = idx - cc * D;
-      const int j = t0 + cc;
-      ks[cc * (D + 1) + d] = j < nB ? kbar[((size_t)bh * nB + j) * D + d] : 0.f;
-    }
-    __syncthreads();
-    float acc[8];
+    float acc[2][4];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+    const float* khead = kbar + ((size_t)bh * nB + t0) * D;
+    for (int d0 = 0; d0 < D; d0 += kDc) {
+      __syncthreads();  // previous slice consumed
+      for (int idx = tid; idx < kRows * kDc; idx += 256) {
+        const int rr = idx / kDc, d = idx - rr * kDc;
+        qs[d * QS + rr] = rr < nrows ? qhead[(size_t)rr * D + d0 + d] : 0.f;
+      }
+      for (int idx = tid; idx < kCols * kDc; idx += 256) {
+        const int cc = idx / kDc, d = idx - cc * kDc;
+        ks[d * KS + cc] = t0 + cc < nB ? khead[(size_t)cc * D + d0 + d] : 0.f;
+      }
+      __syncthreads();
 #pragma unroll 8
-    for (int d = 0; d < D; ++d) {
-      const float qv = qs[rr * (D + 1) + d];
+      for (int d = 0; d < kDc; ++d) {
+        const float q0v = qs[d * QS + 2 * ty], q1v = qs[d * QS + 2 * ty + 1];
+        float kv[4];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) acc[m] = fmaf(qv, ks[(c0 + 8 * m) * (D + 1) + d], acc[m]);
+        for (int c = 0; c < 4; ++c) kv[c] = ks[d * KS + tx + 16 * c];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[0][c] = fmaf(q0v, kv[c], acc[0][c]);
+          acc[1][c] = fmaf(q1v, kv[c], acc[1][c]);
+        }
+      }
     }
 #pragma unroll
-    for (int m = 0; m < 8; ++m) sc[rr * pad + t0 + c0 + 8 * m] = acc[m] * scale;
-    __syncthreads();
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sc[(2 * ty + a) * pad + t0 + tx + 16 * c] = acc[a][c] * scale;
   }
+  __syncthreads();
 
   // row softmax: one warp per row
   for (int r = warp; r < nrows; r += 8) {
@@ -197,7 +217,7 @@ template <int D>
 static cudaError_t launch_scores_d(const float* qbar, const float* kbar, int BH, int nB,
                                    float scale, const int32_t* crp, const int32_t* cc,
                                    float* probs, unsigned* err, cudaStream_t s) {
-  const size_t smem = scores_smem_bytes<D>(nB);
+  const size_t smem = scores_smem_bytes(nB);
   cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -70,8 +70,60 @@ __host__ __device__ __forceinline__ U192 fixed_of_bits(uint32_t bits) {
 
 constexpr unsigned FULL = 0xffffffffu;
 
+// Compare-exchange of the in-register pairs (r, r | J) of a bitonic stage;
+// positions are lane * R + r, and block size k decides the direction.
+template <int J, int R>
+__device__ __forceinline__ void bitonic_in_lane(uint64_t (&key)[R], int lane, int k) {
+  if constexpr (J < R) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if ((r & J) == 0) {
+        const int pr = r | J;
+        const bool desc = ((lane * R + r) & k) == 0;
+        const uint64_t a = key[r], b = key[pr];
+        const bool sw = desc ? (a < b) : (a > b);
+        key[r] = sw ? b : a;
+        key[pr] = sw ? a : b;
+      }
+    }
+  }
+}
+
+// Bitonic sort of 32 * R keys held R per lane, descending; afterwards lane L
+// holds sorted positions L*R .. L*R + R - 1.  The (k, j) stages are runtime
+// loops so the code stays small (a fully unrolled 1024-key network does not
+// fit the instruction cache); register indices stay compile-time constants.
 template <int R>
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void bitonic_sort_desc(uint64_t (&key)[R], int lane) {
+#pragma unroll 1
+  for (int k = 2; k <= 32 * R; k <<= 1) {
+#pragma unroll 1
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= R) {
+        const int lm = j / R;
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint64_t o = __shfl_xor_sync(FULL, key[r], lm);
+          const bool desc = ((lane * R + r) & k) == 0;
+          const bool take_max = lower == desc;
+          key[r] = take_max ? (key[r] > o ? key[r] : o) : (key[r] < o ? key[r] : o);
+        }
+      } else {
+        switch (j) {
+          case 16: bitonic_in_lane<16>(key, lane, k); break;
+          case 8: bitonic_in_lane<8>(key, lane, k); break;
+          case 4: bitonic_in_lane<4>(key, lane, k); break;
+          case 2: bitonic_in_lane<2>(key, lane, k); break;
+          default: bitonic_in_lane<1>(key, lane, k); break;
+        }
+      }
+    }
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(256, 2)
 select_kernel(const float* __restrict__ probs, int rows, int nB, int p_one,
               uint64_t t0, uint64_t t1, uint64_t t2,
               const int32_t* __restrict__ cand_row_ptr, const int32_t* __restrict__ cand_col,
@@ -130,36 +182,7 @@ select_kernel(const float* __restrict__ probs, int rows, int nB, int p_one,
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(FULL, nvalid, o);
 
-  // bitonic sort, descending; lane L holds sorted positions L*R .. L*R+R-1
-#pragma unroll
-  for (int k = 2; k <= 32 * R; k <<= 1) {
-#pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j < R) {
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const int pr = r ^ j;
-          if (pr > r) {
-            const bool desc = ((lane * R + r) & k) == 0;
-            const uint64_t a = key[r], b = key[pr];
-            const bool sw = desc ? (a < b) : (a > b);
-            key[r] = sw ? b : a;
-            key[pr] = sw ? a : b;
-          }
-        }
-      } else {
-        const int lm = j / R;
-        const bool lower = (lane & lm) == 0;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint64_t o = __shfl_xor_sync(FULL, key[r], lm);
-          const bool desc = ((lane * R + r) & k) == 0;
-          const bool take_max = lower == desc;
-          key[r] = take_max ? (key[r] > o ? key[r] : o) : (key[r] < o ? key[r] : o);
-        }
-      }
-    }
-  }
+  bitonic_sort_desc<R>(key, lane);
 
   int kstar = nvalid;
   if (!p_one) {
