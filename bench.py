@@ -30,6 +30,7 @@ import statistics
 import subprocess
 import sys
 import time
+from typing import Tuple
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -153,34 +154,46 @@ class ClockSampler:
                 "power_w_max": max(pw)}
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """Process group from the torchrun environment (one rank per GPU)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
     return world, rank, local
 
 
-def reduce_max(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op: str) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def reduce_max(x: float, world: int) -> float:
+    """Max over ranks (the job's time is its slowest rank's)."""
+    return _reduce(x, world, "max")
 
 
 def reduce_sum(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    """Sum over ranks (each rank runs its own batch)."""
+    return _reduce(x, world, "sum")
+
+
+def job_throughput(local_ms: float, local_flops: float, world: int) -> Tuple[float, float, float]:
+    """(TFLOP/s of the whole job, max step ms over ranks, total FLOPs)."""
+    ms = reduce_max(local_ms, world)
+    flops = reduce_sum(local_flops, world)
+    return flops / (ms * 1e-3) / 1e12, ms, flops
 
 
 def barrier(world: int):
@@ -276,10 +289,11 @@ def config_of(w, args):
 
 def main():
     args = parse_args()
-    world, rank, local = dist_setup()
     if args.impl == "reference":
-        run_reference(args, world, rank)
+        # CPU-only: rank 0 times the oracle, the other ranks leave at once
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
+    world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
@@ -342,10 +356,8 @@ def main():
     t_search = [e[0].elapsed_time(e[1]) for e in ev]
     t_attn = [e[1].elapsed_time(e[2]) for e in ev]
     t_mass = [e[2].elapsed_time(e[3]) for e in ev]
-    ms_step = reduce_max(sum(t_step) / len(t_step), world)
+    value, ms_step, total_flops = job_throughput(sum(t_step) / len(t_step), float(flops), world)
     ms_attn = sum(t_attn) / len(t_attn)
-    total_flops = reduce_sum(float(flops), world)
-    value = total_flops / (ms_step * 1e-3) / 1e12
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12
     peaks = measured_peaks()
 
@@ -373,6 +385,8 @@ def main():
                     "executed_tflop": flops / 1e12, "dense_tflop": dense_flops / 1e12}
     line["clocks"] = clk
 
+    out_ref = out.clone()  # the p-run's O, before the dense run reuses `out`
+
     # dense p = 1 reference: the same kernel over an all-blocks CSR
     if not args.no_dense:
         rp_all = (torch.arange(rows + 1, device=dev, dtype=torch.int64) * nB).to(torch.int32)
@@ -396,24 +410,30 @@ def main():
         }
         del rp_all, col_all
 
-    # end to end through the public calls with pinned host buffers
+    # end to end through the public host-buffer call: pinned Q, K, V in, O out,
+    # with the PCIe copies of one chunk of heads overlapping another's compute
     if not args.no_e2e:
+        from dynamic_block_sparse_pool_b200.pipeline import HostPipeline
         qh, kh, vh = q_c.pin_memory(), k_c.pin_memory(), v_c.pin_memory()
-        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        ke = max(2, args.steps // 2)
+        oh = torch.empty(q_c.shape, dtype=q_c.dtype).pin_memory()
+        del P, ws_pool, ws_sel, col_idx, blk_lse, mass  # make room for the pipeline's slots
+        torch.cuda.empty_cache()
+        pipe = HostPipeline(B, H, N, D, w.dtype, blk)
+        ke = max(2, args.steps // 3)
         ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(ke + 1)]
-        for s in range(ke + 1):  # first iteration is a warm-up
-            ee[s][0].record(stream)
-            q.copy_(qh, non_blocking=True); k.copy_(kh, non_blocking=True); v.copy_(vh, non_blocking=True)
-            search(); attend(); finish()
-            oh.copy_(out, non_blocking=True)
-            ee[s][1].record(stream)
+        for s_ in range(ke + 1):  # first iteration is a warm-up
+            ee[s_][0].record(stream)
+            pipe.run(qh, kh, vh, oh, args.p, scale)
+            ee[s_][1].record(stream)
         torch.cuda.synchronize(dev)
         ms_e2e = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ee[1:]) / ke, world)
         line["e2e"] = {"value": total_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-                       "ms_per_step": ms_e2e,
-                       "h2d_bytes_per_step": 3 * q_c.numel() * q_c.element_size(),
-                       "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+                       "ms_per_step": ms_e2e, "api": "pipeline.HostPipeline.run",
+                       "chunk_heads": pipe.chunk,
+                       "h2d_bytes_per_step": pipe.h2d_bytes(),
+                       "d2h_bytes_per_step": pipe.d2h_bytes()}
+        # the chunked host run must reproduce the device-resident run bit for bit
+        line["e2e"]["matches_device_run"] = bool(torch.equal(oh.to(dev), out_ref))
 
     if rank == 0 and world == 1 and not args.no_cpu:
         val, desc, threads, _ = oracle_sample(w, q_c, k_c, v_c, args.p, args.cpu_seconds)
