@@ -46,7 +46,10 @@ ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn
 # DRAM bytes per attention launch from an ncu capture, keyed by the sha256
 # prefix of attn_sm100.cu at capture time (scaled to the full workload when
 # the capture ran a smaller case); stale entries are ignored.
-ATTN_TRAFFIC = {}
+ATTN_TRAFFIC = {
+    # 8-head Wan2.1-like capture: 539.9 MB read + 498.3 MB written, x5 heads
+    "05cc2902bc8dc9ae": int((539873792 + 498344960) * 5),
+}
 
 
 def parse_args():
@@ -63,6 +66,9 @@ def parse_args():
     ap.add_argument("--no-dense", action="store_true", help="skip the p=1 reference run")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the bench line: one JSON line per point of the "
+                         "p-sweep, reduced search, HunyuanVideo schedule and CogVideoX runs")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -285,6 +291,101 @@ def config_of(w, args):
             "l2": "inputs larger than L2 (Q,K,V %.2f GB)" % (3 * w.BH * w.N * w.head_dim * 2 / 1e9)}
 
 
+
+# --------------------------------------------------------------------- sweep --
+
+def sweep(args):
+    """Timing of the measurement plan's points, one JSON line each."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, reps):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream); fn(); b.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in ev) / reps
+
+    def point(w, q, k, v, p, cand=None, dense_ms=None, label=None, extra=None):
+        B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+        nB, rows = w.n_blocks, w.BH * w.n_blocks
+        scale = 1.0 / math.sqrt(D)
+        P = torch.empty(B * H, nB, nB, device=dev)
+        wp = torch.empty(ops.workspace_size(0, B, H, N, D, blk), device=dev, dtype=torch.uint8)
+        wsel = torch.empty(ops.workspace_size(1, B, H, N, D, blk), device=dev, dtype=torch.uint8)
+        rp = torch.empty(rows + 1, device=dev, dtype=torch.int32)
+        ci = torch.empty(rows * nB, device=dev, dtype=torch.int32)
+        out = torch.empty_like(q)
+        lse = torch.empty(B, H, N, device=dev)
+        cap = rows * nB if cand is None else int(cand[0][-1])
+        bl = torch.empty(max(cap, 1), blk, device=dev)
+        ms_ = torch.empty(max(cap, 1), device=dev)
+        search = lambda: (ops.pool_score(q, k, blk, scale, cand=cand, out=P, workspace=wp),
+                          ops.select_topp(P, p, cand=cand, row_ptr=rp, col_idx=ci, workspace=wsel))
+        attend = lambda: ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=bl)
+        mass = lambda: ops.block_mass(lse, bl, rp, blk, mass=ms_)
+        search(); attend(); mass(); ops.device_status(dev)
+        flops, nnz = executed_flops(rp, ci, N, blk, D, nB)
+        reps = 5
+        t_s = timed(search, reps)
+        t_a = timed(attend, reps)
+        t_m = timed(mass, reps)
+        step = t_s + t_a + t_m
+        line = {"sweep": label or w.name, "p": p, "reduced_search": cand is not None,
+                "density": nnz / (rows * nB), "executed_tflop": flops / 1e12,
+                "search_ms": t_s, "attn_ms": t_a, "mass_ms": t_m, "step_ms": step,
+                "attn_tflops": flops / (t_a * 1e-3) / 1e12,
+                "step_tflops": flops / (step * 1e-3) / 1e12}
+        if dense_ms is not None:
+            red = (4 * D * B * H * N * N) / flops
+            line.update({"dense_attn_ms": dense_ms, "flop_reduction": red,
+                         "speedup_attn": dense_ms / t_a, "speedup_pipeline": dense_ms / step,
+                         "pipeline_over_reduction": dense_ms / step / red})
+        if extra:
+            line.update(extra)
+        print(json.dumps(line), flush=True)
+        return rp[: rows + 1].clone(), ci[:nnz].clone(), line
+
+    def dense_ms_of(w, q, k, v):
+        B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+        nB, rows = w.n_blocks, w.BH * w.n_blocks
+        rpa = (torch.arange(rows + 1, device=dev, dtype=torch.int64) * nB).to(torch.int32)
+        cia = torch.arange(nB, device=dev, dtype=torch.int32).repeat(rows)
+        out = torch.empty_like(q)
+        f = lambda: ops.attn_fwd(q, k, v, rpa, cia, blk, 1.0 / math.sqrt(D), out=out,
+                                 want_lse=False, want_blk_lse=False)
+        f(); torch.cuda.synchronize(dev)
+        return timed(f, 3)
+
+    # Wan2.1-like: p sweep, then reduced search
+    w = synth.WAN21
+    q, k, v = synth.make_qkv(w, 0, device="cuda")
+    dms = dense_ms_of(w, q, k, v)
+    masks = {}
+    for p in w.p:
+        masks[p] = point(w, q, k, v, p, dense_ms=dms)[:2]
+    q1, k1, v1 = synth.make_qkv(w, 1, device="cuda")
+    dms1 = dense_ms_of(w, q1, k1, v1)
+    point(w, q1, k1, v1, 0.7, dense_ms=dms1, label=w.name + " seed1 full search")
+    point(w, q1, k1, v1, 0.7, cand=masks[0.95], dense_ms=dms1,
+          label=w.name + " seed1 reduced search (candidates: seed0 p=0.95 mask)")
+    del q, k, v, q1, k1, v1
+    torch.cuda.empty_cache()
+    # HunyuanVideo-like growing-sparsity schedule
+    w = synth.HUNYUAN
+    for step, p, bw, seed in synth.hunyuan_schedule(10):
+        q, k, v = synth.make_qkv(w, seed, bandwidth=bw, device="cuda")
+        dms = dense_ms_of(w, q, k, v) if step in (0, 9) else None
+        point(w, q, k, v, round(p, 4), dense_ms=dms, label=f"{w.name} step {step}",
+              extra={"bandwidth": bw, "seed": seed})
+        del q, k, v
+    # CogVideoX-like
+    w = synth.COGVIDEOX
+    q, k, v = synth.make_qkv(w, 0, device="cuda")
+    point(w, q, k, v, 0.9, dense_ms=dense_ms_of(w, q, k, v))
+
 # ---------------------------------------------------------------- GPU bench --
 
 def main():
@@ -292,6 +393,9 @@ def main():
     if args.impl == "reference":
         # CPU-only: rank 0 times the oracle, the other ranks leave at once
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    if args.sweep:
+        sweep(args)
         return
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)

@@ -129,37 +129,41 @@ def lengthscales(w: Workload, bandwidth: float) -> torch.Tensor:
 
 
 def make_qkv(w: Workload, seed: int, bandwidth: Optional[float] = None,
-             heads: Optional[Sequence[int]] = None):
+             heads: Optional[Sequence[int]] = None, device: str = "cpu"):
     """Draw (q, k, v), each [B, H, N, D] in ``w.dtype``, on the CPU.
 
     ``heads`` restricts the draw to a subset of heads (same values as the
     full draw for those heads: every head has its own generator stream).
+    ``device="cuda"`` draws with the same recipe on the GPU (a different
+    random stream, so different values with the same distribution): for
+    timing runs that need many large inputs, not for comparisons with a
+    CPU draw.
     """
     bw = w.bandwidth if bandwidth is None else bandwidth
-    coords = (grid_coords(w.T, w.Hg, w.W) / lengthscales(w, bw)).to(torch.float32)
+    coords = (grid_coords(w.T, w.Hg, w.W) / lengthscales(w, bw)).to(torch.float32).to(device)
     D, N, P = w.head_dim, w.N, w.n_prefix
     head_ids = list(range(w.heads)) if heads is None else list(heads)
     shape = (w.batch, len(head_ids), N, D)
-    q = torch.empty(shape, dtype=w.dtype)
-    k = torch.empty(shape, dtype=w.dtype)
-    v = torch.empty(shape, dtype=w.dtype)
+    q = torch.empty(shape, dtype=w.dtype, device=device)
+    k = torch.empty(shape, dtype=w.dtype, device=device)
+    v = torch.empty(shape, dtype=w.dtype, device=device)
     for b in range(w.batch):
         for hi, h in enumerate(head_ids):
-            g = torch.Generator().manual_seed(
+            g = torch.Generator(device=device).manual_seed(
                 (seed * 1000003 + b * 1009 + h) & 0x7FFFFFFF)
-            omega = torch.randn(D, 3, generator=g)
-            beta = torch.rand(D, generator=g) * (2.0 * math.pi)
+            omega = torch.randn(D, 3, generator=g, device=device)
+            beta = torch.rand(D, generator=g, device=device) * (2.0 * math.pi)
             phi = math.sqrt(2.0) * torch.cos(coords @ omega.T + beta)
-            qh = torch.empty(N, D)
-            kh = torch.empty(N, D)
-            qh[P:] = 0.7 * phi + 0.5 * torch.randn(N - P, D, generator=g)
-            kh[P:] = 0.7 * phi + 0.5 * torch.randn(N - P, D, generator=g)
+            qh = torch.empty(N, D, device=device)
+            kh = torch.empty(N, D, device=device)
+            qh[P:] = 0.7 * phi + 0.5 * torch.randn(N - P, D, generator=g, device=device)
+            kh[P:] = 0.7 * phi + 0.5 * torch.randn(N - P, D, generator=g, device=device)
             if P:
-                qh[:P] = torch.randn(P, D, generator=g)
-                kh[:P] = torch.randn(P, D, generator=g)
-            sinks = torch.randint(0, N, (w.n_sinks,), generator=g)
+                qh[:P] = torch.randn(P, D, generator=g, device=device)
+                kh[:P] = torch.randn(P, D, generator=g, device=device)
+            sinks = torch.randint(0, N, (w.n_sinks,), generator=g, device=device)
             kh[sinks] += 3.0 * qh.mean(0)
-            vh = torch.randn(N, D, generator=g)
+            vh = torch.randn(N, D, generator=g, device=device)
             q[b, hi] = qh.to(w.dtype)
             k[b, hi] = kh.to(w.dtype)
             v[b, hi] = vh.to(w.dtype)
