@@ -122,19 +122,124 @@ __device__ __forceinline__ void bitonic_sort_desc(uint64_t (&key)[R], int lane) 
   }
 }
 
+// Level of a probability for the threshold search: its exponent and the top
+// three mantissa bits (values within 12.5 % share a level).  Probabilities
+// are in [0, 1], so levels run from 0 to 1016.
+__device__ __forceinline__ int level_of(uint32_t bits) { return (int)(bits >> 20); }
+constexpr int kLevels = 1017;
+
+__device__ __forceinline__ U192 warp_sum192(U192 v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    U192 o;
+    o.w0 = __shfl_xor_sync(FULL, v.w0, off);
+    o.w1 = __shfl_xor_sync(FULL, v.w1, off);
+    o.w2 = __shfl_xor_sync(FULL, v.w2, off);
+    add192(v, o);
+  }
+  return v;
+}
+
 template <int R>
-__global__ void __launch_bounds__(256, 2)
+__device__ __forceinline__ double level_sum_f64(const uint32_t (&bits)[R], uint32_t valid, int lv) {
+  double s = 0.0;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (((valid >> r) & 1u) && level_of(bits[r]) >= lv) s += (double)__uint_as_float(bits[r]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(FULL, s, off);
+  return s;
+}
+
+// Sorts the n boundary keys of a warp (in shared memory) descending and
+// returns how many of them, taken in order, first bring the running exact
+// sum `base` to `target` (n if none does).  R = keys per lane.
+template <int R>
+__device__ __noinline__ int boundary_cut(uint64_t* keys, int n, U192 base, const U192 target,
+                                         int lane) {
+  uint64_t key[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int i = lane * R + r;
+    key[r] = i < n ? keys[i] : 0ull;
+  }
+  bitonic_sort_desc<R>(key, lane);
+  U192 own{0ull, 0ull, 0ull};
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (key[r]) add192(own, fixed_of_bits((uint32_t)(key[r] >> 32) - 1u));
+  U192 incl = own;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    U192 o;
+    o.w0 = __shfl_up_sync(FULL, incl.w0, off);
+    o.w1 = __shfl_up_sync(FULL, incl.w1, off);
+    o.w2 = __shfl_up_sync(FULL, incl.w2, off);
+    if (lane >= off) add192(incl, o);
+  }
+  U192 excl;
+  excl.w0 = __shfl_up_sync(FULL, incl.w0, 1);
+  excl.w1 = __shfl_up_sync(FULL, incl.w1, 1);
+  excl.w2 = __shfl_up_sync(FULL, incl.w2, 1);
+  if (lane == 0) excl = U192{0ull, 0ull, 0ull};
+  U192 ti = incl;
+  add192(ti, base);
+  const unsigned ball = __ballot_sync(FULL, ge192(ti, target));
+  int cut = n;
+  if (ball) {
+    const int L = __ffs(ball) - 1;
+    int kk = 0;
+    if (lane == L) {
+      U192 acc = excl;
+      add192(acc, base);
+      bool done = false;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (!done && key[r]) {
+          add192(acc, fixed_of_bits((uint32_t)(key[r] >> 32) - 1u));
+          if (ge192(acc, target)) {
+            kk = L * R + r + 1;
+            done = true;
+          }
+        }
+      }
+    }
+    cut = __shfl_sync(FULL, kk, L);
+  }
+  // write the sorted order back so the caller can mark the first `cut`
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int i = lane * R + r;
+    if (i < n) keys[i] = key[r];
+  }
+  __syncwarp();
+  return cut;
+}
+
+// One warp per row: values of up to 32 * R candidate blocks, R per lane
+// (element e = r * 32 + lane).
+//   1. A binary search over levels, with fp64 sums (exact to ~1e-13), finds
+//      the level t where the mass of everything at or above t first reaches p.
+//   2. An exact 192-bit pass verifies mass(level > t) < p <= mass(level >= t)
+//      and moves t by one level if rounding misled the search.
+//   3. Everything above level t is kept.  The few blocks on level t are
+//      sorted by (probability desc, index asc) and kept until the exact sum
+//      reaches p.
+template <int R>
+__global__ void __launch_bounds__(128)
 select_kernel(const float* __restrict__ probs, int rows, int nB, int p_one,
               uint64_t t0, uint64_t t1, uint64_t t2,
               const int32_t* __restrict__ cand_row_ptr, const int32_t* __restrict__ cand_col,
               uint32_t* __restrict__ bitmaps, int32_t* __restrict__ counts, unsigned* err) {
-  __shared__ uint32_t cbits_all[8][32];
-  __shared__ uint32_t sel_all[8][32];
+  __shared__ uint32_t cbits_all[4][32];
+  __shared__ uint32_t sel_all[4][32];
+  __shared__ uint64_t bkeys_all[4][32 * R];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
+  const int row = blockIdx.x * 4 + warp;
   if (row >= rows) return;  // whole warp leaves together
   uint32_t* cbits = cbits_all[warp];
   uint32_t* sel = sel_all[warp];
+  uint64_t* bkeys = bkeys_all[warp];
   const bool reduced = cand_row_ptr != nullptr;
   const U192 target{t0, t1, t2};
 
@@ -158,84 +263,116 @@ select_kernel(const float* __restrict__ probs, int rows, int nB, int p_one,
   }
   __syncwarp();
 
-  // keys: ((prob bits + 1) << 32) | ~index for candidates, 0 otherwise;
-  // larger key = earlier in the (prob desc, index asc) order
   const float* prow = probs + (size_t)row * nB;
-  uint64_t key[R];
-  int nvalid = 0;
+  uint32_t bits[R];
+  uint32_t valid = 0u;  // bit r: element r * 32 + lane is a candidate
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int e = r * 32 + lane;
-    uint64_t kv = 0ull;
+    bits[r] = 0u;
     if (e < nB && (!reduced || ((cbits[e >> 5] >> (e & 31)) & 1u))) {
       float f = prow[e];
       if (!(f >= 0.f && f <= 1.f)) {
         flag_error(err, kErrProb);
         f = 0.f;
       }
-      const uint32_t bits = __float_as_uint(f) & 0x7FFFFFFFu;
-      kv = ((uint64_t)(bits + 1u) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
-      ++nvalid;
+      bits[r] = __float_as_uint(f) & 0x7FFFFFFFu;
+      valid |= 1u << r;
     }
-    key[r] = kv;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(FULL, nvalid, o);
 
-  bitonic_sort_desc<R>(key, lane);
-
-  int kstar = nvalid;
+  int kstar_extra = 0;  // boundary blocks kept (only when cut inside a level)
+  int t_level = -1;     // keep everything with level > t_level (-1: keep all)
+  int n_bnd = 0;
   if (!p_one) {
-    U192 own{0ull, 0ull, 0ull};
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-      if (key[r]) add192(own, fixed_of_bits((uint32_t)(key[r] >> 32) - 1u));
-    U192 incl = own;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      U192 o;
-      o.w0 = __shfl_up_sync(FULL, incl.w0, off);
-      o.w1 = __shfl_up_sync(FULL, incl.w1, off);
-      o.w2 = __shfl_up_sync(FULL, incl.w2, off);
-      if (lane >= off) add192(incl, o);
+    // 1. threshold level from fp64 sums: largest t with mass(level >= t) >= p
+    const double tgt = ldexp((double)t0, -149) + ldexp((double)t1, -85) + ldexp((double)t2, -21);
+    int lo = -1, hi = kLevels;  // invariant: mass(>= lo) >= p (lo = -1: all), mass(>= hi) < p
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (level_sum_f64<R>(bits, valid, mid) >= tgt) lo = mid;
+      else hi = mid;
     }
-    U192 excl;
-    excl.w0 = __shfl_up_sync(FULL, incl.w0, 1);
-    excl.w1 = __shfl_up_sync(FULL, incl.w1, 1);
-    excl.w2 = __shfl_up_sync(FULL, incl.w2, 1);
-    if (lane == 0) excl = U192{0ull, 0ull, 0ull};
-    const unsigned ball = __ballot_sync(FULL, ge192(incl, target));
-    if (ball) {
-      const int L = __ffs(ball) - 1;
-      int kk = 0;
-      if (lane == L) {
-        U192 acc = excl;
-        bool done = false;
+    // 2. exact check of mass(level > t) < p <= mass(level >= t); fix by a level
+    int t = lo;
+    // each correction moves t one level towards the exact answer, so the loop
+    // ends; fp64 sums of at most 1024 non-negative terms are off by ~1e-13,
+    // which moves t by at most one level in practice
+    for (int guard = 0; guard <= kLevels + 1; ++guard) {
+      U192 above{0ull, 0ull, 0ull}, at_or_above{0ull, 0ull, 0ull};
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          if (!done && key[r]) {
-            add192(acc, fixed_of_bits((uint32_t)(key[r] >> 32) - 1u));
-            if (ge192(acc, target)) {
-              kk = L * R + r + 1;
-              done = true;
-            }
+      for (int r = 0; r < R; ++r) {
+        if ((valid >> r) & 1u) {
+          const int lv = level_of(bits[r]);
+          if (lv >= t) {
+            const U192 x = fixed_of_bits(bits[r]);
+            add192(at_or_above, x);
+            if (lv > t) add192(above, x);
           }
         }
       }
-      kstar = __shfl_sync(FULL, kk, L);
+      above = warp_sum192(above);
+      at_or_above = warp_sum192(at_or_above);
+      if (t >= 0 && !ge192(at_or_above, target)) {
+        --t;  // the fp64 search stopped one level too high
+        continue;
+      }
+      if (ge192(above, target)) {
+        ++t;  // one level too low
+        continue;
+      }
+      // 3. blocks on level t, compacted in index order, then sorted and cut
+      if (t >= 0) {
+        int mine = 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (((valid >> r) & 1u) && level_of(bits[r]) == t) ++mine;
+        int incl = mine;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int o = __shfl_up_sync(FULL, incl, off);
+          if (lane >= off) incl += o;
+        }
+        n_bnd = __shfl_sync(FULL, incl, 31);
+        int pos = incl - mine;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (((valid >> r) & 1u) && level_of(bits[r]) == t)
+            bkeys[pos++] = ((uint64_t)(bits[r] + 1u) << 32) |
+                           (uint64_t)(0xFFFFFFFFu - (uint32_t)(r * 32 + lane));
+        __syncwarp();
+        const int rb = (n_bnd + 31) / 32;
+        if (rb <= 1) kstar_extra = boundary_cut<1>(bkeys, n_bnd, above, target, lane);
+        else if (rb <= 2) kstar_extra = boundary_cut<2 <= R ? 2 : R>(bkeys, n_bnd, above, target, lane);
+        else if (rb <= 4) kstar_extra = boundary_cut<4 <= R ? 4 : R>(bkeys, n_bnd, above, target, lane);
+        else if (rb <= 8) kstar_extra = boundary_cut<8 <= R ? 8 : R>(bkeys, n_bnd, above, target, lane);
+        else if (rb <= 16) kstar_extra = boundary_cut<16 <= R ? 16 : R>(bkeys, n_bnd, above, target, lane);
+        else kstar_extra = boundary_cut<R>(bkeys, n_bnd, above, target, lane);
+      }
+      t_level = t;
+      break;
     }
   }
 
+  // keep: level > t_level, plus the first kstar_extra sorted boundary blocks
+  int kept = 0;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    if (lane * R + r < kstar && key[r]) {
-      const uint32_t e = 0xFFFFFFFFu - (uint32_t)key[r];
+    if (((valid >> r) & 1u) && level_of(bits[r]) > t_level) {
+      const int e = r * 32 + lane;
       atomicOr(&sel[e >> 5], 1u << (e & 31));
+      ++kept;
     }
   }
+  for (int i = lane; i < kstar_extra; i += 32) {
+    const uint32_t e = 0xFFFFFFFFu - (uint32_t)bkeys[i];
+    atomicOr(&sel[e >> 5], 1u << (e & 31));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(FULL, kept, o);
   __syncwarp();
   bitmaps[(size_t)row * 32 + lane] = sel[lane];
-  if (lane == 0) counts[row] = kstar;
+  if (lane == 0) counts[row] = kept + kstar_extra;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -325,10 +462,11 @@ cudaError_t launch_select(const float* probs, int rows, int nB, float p,
   const int grid = ceil_div(rows, 8);
   const int R = nB <= 32 ? 1 : nB <= 64 ? 2 : nB <= 128 ? 4 : nB <= 256 ? 8 : nB <= 512 ? 16 : 32;
   switch (R) {
-#define DSA_SEL(RR)                                                                        \
-  case RR:                                                                                 \
-    select_kernel<RR><<<grid, 256, 0, s>>>(probs, rows, nB, p_one, t.w0, t.w1, t.w2,       \
-                                           cand_row_ptr, cand_col, bitmaps, counts, err);  \
+#define DSA_SEL(RR)                                                                            \
+  case RR:                                                                                     \
+    select_kernel<RR><<<ceil_div(rows, 4), 128, 0, s>>>(probs, rows, nB, p_one, t.w0, t.w1,   \
+                                                        t.w2, cand_row_ptr, cand_col, bitmaps, \
+                                                        counts, err);                          \
     break;
     DSA_SEL(1) DSA_SEL(2) DSA_SEL(4) DSA_SEL(8) DSA_SEL(16) DSA_SEL(32)
 #undef DSA_SEL
