@@ -9,10 +9,10 @@
 // Kernel 1 (pool_means): one CTA per (block, head, Q-or-K); 16-byte loads,
 //   fp32 accumulation, mean over the block's actual rows.  HBM-bound: reads
 //   Q and K once.
-// Kernel 2 (block_scores): one CTA per (32 query-block rows, head): a
-//   register-tiled fp32 product of the 32 pooled queries with tiles of 64
-//   pooled keys; the 32 x nB raw scores stay in shared memory for the row
-//   softmax, which writes P once, coalesced.
+// Kernel 2 (block_scores): one CTA per (64 query-block rows, head): a
+//   register-tiled fp32 product of the 64 pooled queries with double-buffered
+//   tiles of 64 pooled keys (cp.async), scaled scores written to P with a
+//   running max and sum per row, then P normalised in place from L2.
 #include "common.cuh"
 
 namespace dsa {
@@ -57,46 +57,86 @@ pool_means_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int n
   }
 }
 
-constexpr int kRows = 32;   // query-block rows per CTA
-constexpr int kCols = 64;   // key blocks per score tile
-constexpr int kDc = 32;     // head-dim slice staged in shared memory at a time
+constexpr int kTile = 64;  // query-block rows per CTA and key blocks per score tile
 
-__host__ __device__ constexpr int scores_pad(int nB) { return ceil_div(nB, kCols) * kCols; }
-
-__host__ __device__ constexpr size_t scores_smem_bytes(int nB) {
-  return sizeof(float) * ((size_t)kDc * (kRows + 1) + (size_t)kDc * (kCols + 1) +
-                          (size_t)kRows * scores_pad(nB)) +
-         sizeof(uint32_t) * kRows * 32;
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Scores of 32 pooled queries against all pooled keys of a head, then the row
-// softmax.  The 32 x 64 score tile is a register-tiled fp32 product: thread
-// (ty, tx) of a 16 x 16 grid computes rows 2*ty, 2*ty+1 and columns
-// tx + 16*c (c < 4): 6 shared-memory loads per 8 FMAs, from transposed
-// slices of 32 head dimensions padded to odd strides (conflict-free both when
-// staged and when read).
+// Shared memory of the score kernel: the CTA's 64 pooled queries, a double
+// buffer of 64 pooled keys (rows padded to D + 4 floats: 16-byte aligned, and
+// each quarter-warp's float4 reads fall in distinct banks), the candidate
+// bitmaps and the per-row softmax statistics.
 template <int D>
-__global__ void __launch_bounds__(256)
+struct ScoreSmem {
+  static constexpr int kStride = D + 4;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTile * kStride;          // floats
+  static constexpr int kBits = kK + 2 * kTile * kStride;   // floats -> uint32 [64][32]
+  static constexpr int kStat = kBits + kTile * 32;         // float2 [64]
+  static constexpr size_t kBytes = sizeof(float) * (size_t)(kStat + 2 * kTile);
+};
+
+// Copies `count` rows (count >= 1) of D floats starting at row `first` into a
+// 64-row tile; rows past `count` repeat the last row (their scores are never
+// used).
+template <int D>
+__device__ __forceinline__ void stage_rows(float* dst, const float* src, int first, int count,
+                                           int tid) {
+  constexpr int C = D / 4;  // 16-byte chunks per row
+#pragma unroll 2
+  for (int c = tid; c < kTile * C; c += 256) {
+    const int r = c / C, q4 = c - r * C;
+    const int rr = min(r, count - 1);
+    cp_async16(dst + r * ScoreSmem<D>::kStride + q4 * 4, src + (size_t)(first + rr) * D + q4 * 4);
+  }
+}
+
+// Softmax over the key blocks of scale * qbar_i . kbar_j for 64 query blocks
+// of one head (all key blocks, or the candidate set of each row).
+//   Pass 1: 64 x 64 score tiles, thread (ty, tx) of a 16 x 16 grid holding
+//     rows 4ty .. 4ty+3 and columns tx + 16c (c < 4), fp32 FMAs over the
+//     head dimension.  The scaled scores go to P as they are; each thread
+//     keeps a running (max, sum of exp) per row, merged across the 16
+//     threads of a row at the end.
+//   Pass 2: one warp per row rewrites P as exp(s - max) / sum (reads hit L2:
+//     the CTA wrote them just before).  Non-candidates and empty rows get 0.
+template <int D>
+__global__ void __launch_bounds__(256, 2)
 block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                     int nB, float scale, const int32_t* __restrict__ cand_row_ptr,
                     const int32_t* __restrict__ cand_col, float* __restrict__ probs,
                     unsigned* err) {
-  extern __shared__ float sm[];
-  constexpr int QS = kRows + 1, KS = kCols + 1;    // padded strides
-  float* qs = sm;                                  // [kDc][QS]   (transposed)
-  float* ks = qs + kDc * QS;                       // [kDc][KS]   (transposed)
-  float* sc = ks + kDc * KS;                       // [kRows][pad]
-  const int pad = scores_pad(nB);
-  uint32_t* cbits = reinterpret_cast<uint32_t*>(sc + kRows * pad);  // [kRows][32]
+  using L = ScoreSmem<D>;
+  constexpr int S = L::kStride;
+  extern __shared__ __align__(16) float sm[];
+  float* qs = sm + L::kQ;
+  float* ks = sm + L::kK;
+  uint32_t* cbits = reinterpret_cast<uint32_t*>(sm + L::kBits);  // [64][32]
+  float2* stat = reinterpret_cast<float2*>(sm + L::kStat);       // [64]
+  __shared__ uint32_t live_tiles;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ty = tid >> 4, tx = tid & 15;
   const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kRows;
-  const int nrows = min(kRows, nB - i0);
+  const int i0 = blockIdx.x * kTile;
+  const int nrows = min(kTile, nB - i0);
+  const int n_tiles = ceil_div(nB, kTile);
   const bool reduced = cand_row_ptr != nullptr;
+  const float* khead = kbar + (size_t)bh * nB * D;
 
+  stage_rows<D>(qs, qbar + (size_t)bh * nB * D, i0, nrows, tid);
+  cp_async_commit();
+
+  if (tid == 0) live_tiles = reduced ? 0u : (n_tiles >= 32 ? 0xFFFFFFFFu : (1u << n_tiles) - 1u);
   if (reduced) {
-    for (int idx = tid; idx < kRows * 32; idx += 256) cbits[idx] = 0u;
+    for (int idx = tid; idx < kTile * 32; idx += 256) cbits[idx] = 0u;
     __syncthreads();
     for (int rr = warp; rr < nrows; rr += 8) {
       const size_t row = (size_t)bh * nB + i0 + rr;
@@ -114,81 +154,128 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
         atomicOr(&cbits[rr * 32 + (j >> 5)], 1u << (j & 31));
       }
     }
+    __syncthreads();
+    // tiles holding a candidate of any of the CTA's rows (word w covers tile w / 2)
+    uint32_t mine = 0u;
+    for (int rr = warp; rr < nrows; rr += 8)
+      if (cbits[rr * 32 + lane]) mine |= 1u << (lane >> 1);
+    mine = __reduce_or_sync(0xffffffffu, mine);
+    if (lane == 0 && mine) atomicOr(&live_tiles, mine);
   }
   __syncthreads();
+  uint32_t live = live_tiles;
 
-  const int ty = tid >> 4, tx = tid & 15;
-  const float* qhead = qbar + ((size_t)bh * nB + i0) * D;
-  for (int t0 = 0; t0 < nB; t0 += kCols) {
-    if (reduced) {
-      // skip a tile that holds no candidate of any of this CTA's rows
-      bool any = false;
-      if (tid < 64) {
-        const int w = (t0 >> 5) + (tid >> 5);
-        any = w < 32 && cbits[(tid & 31) * 32 + w] != 0u;
-      }
-      if (!__syncthreads_or(any)) continue;
-    }
-    float acc[2][4];
+  float run_m[4], run_s[4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 4; ++a) {
+    run_m[a] = -INFINITY;
+    run_s[a] = 0.f;
+  }
+  float* prow_base = probs + ((size_t)bh * nB + i0) * nB;
+
+  int t = live ? __ffs(live) - 1 : n_tiles;
+  if (t < n_tiles) stage_rows<D>(ks, khead, t * kTile, min(kTile, nB - t * kTile), tid);
+  cp_async_commit();
+  for (int buf = 0; t < n_tiles; buf ^= 1) {
+    live &= ~(1u << t);
+    const int tn = live ? __ffs(live) - 1 : n_tiles;
+    if (tn < n_tiles)
+      stage_rows<D>(ks + (buf ^ 1) * kTile * S, khead, tn * kTile, min(kTile, nB - tn * kTile), tid);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+
+    const float* kt = ks + buf * kTile * S;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-    const float* khead = kbar + ((size_t)bh * nB + t0) * D;
-    for (int d0 = 0; d0 < D; d0 += kDc) {
-      __syncthreads();  // previous slice consumed
-      for (int idx = tid; idx < kRows * kDc; idx += 256) {
-        const int rr = idx / kDc, d = idx - rr * kDc;
-        qs[d * QS + rr] = rr < nrows ? qhead[(size_t)rr * D + d0 + d] : 0.f;
-      }
-      for (int idx = tid; idx < kCols * kDc; idx += 256) {
-        const int cc = idx / kDc, d = idx - cc * kDc;
-        ks[d * KS + cc] = t0 + cc < nB ? khead[(size_t)cc * D + d0 + d] : 0.f;
-      }
-      __syncthreads();
-#pragma unroll 8
-      for (int d = 0; d < kDc; ++d) {
-        const float q0v = qs[d * QS + 2 * ty], q1v = qs[d * QS + 2 * ty + 1];
-        float kv[4];
+#pragma unroll 2
+    for (int d = 0; d < D; d += 4) {
+      float4 qv[4], kv[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) kv[c] = ks[d * KS + tx + 16 * c];
+      for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qs + (4 * ty + a) * S + d);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(kt + (tx + 16 * c) * S + d);
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          acc[0][c] = fmaf(q0v, kv[c], acc[0][c]);
-          acc[1][c] = fmaf(q1v, kv[c], acc[1][c]);
+          acc[a][c] = fmaf(qv[a].x, kv[c].x, acc[a][c]);
+          acc[a][c] = fmaf(qv[a].y, kv[c].y, acc[a][c]);
+          acc[a][c] = fmaf(qv[a].z, kv[c].z, acc[a][c]);
+          acc[a][c] = fmaf(qv[a].w, kv[c].w, acc[a][c]);
+        }
+    }
+
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = 4 * ty + a;
+      float x[4];
+      bool ok[4];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = t * kTile + tx + 16 * c;
+        x[c] = acc[a][c] * scale;
+        ok[c] = r < nrows && j < nB && (!reduced || ((cbits[r * 32 + (j >> 5)] >> (j & 31)) & 1u));
+        if (ok[c]) {
+          prow_base[(size_t)r * nB + j] = x[c];
+          mx = fmaxf(mx, x[c]);
         }
       }
+      if (mx > run_m[a]) {
+        run_s[a] = run_m[a] == -INFINITY ? 0.f : run_s[a] * expf(run_m[a] - mx);
+        run_m[a] = mx;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (ok[c]) run_s[a] += expf(x[c] - run_m[a]);
     }
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) sc[(2 * ty + a) * pad + t0 + tx + 16 * c] = acc[a][c] * scale;
+    __syncthreads();  // this buffer is refilled two tiles later
+    t = tn;
   }
-  __syncthreads();
+  cp_async_wait<0>();
 
-  // row softmax: one warp per row
+  // merge the 16 partial (max, sum) of each row: lanes tx of one half-warp
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    float m = run_m[a], s = run_s[a];
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+      const float so = __shfl_xor_sync(0xffffffffu, s, o);
+      const float M = fmaxf(m, mo);
+      s = (m == -INFINITY ? 0.f : s * expf(m - M)) + (mo == -INFINITY ? 0.f : so * expf(mo - M));
+      m = M;
+    }
+    if (tx == 0) stat[4 * ty + a] = make_float2(m, s);
+  }
+  __syncthreads();  // also orders pass 1's global writes before pass 2's reads
+
+  // 16 independent loads per lane in flight (the reads come from L2)
+  constexpr int kU = 16;
   for (int r = warp; r < nrows; r += 8) {
+    const float2 ms = stat[r];
+    const bool empty = !(ms.x > -INFINITY);
     const uint32_t* bits = cbits + r * 32;
-    float* srow = sc + r * pad;
-    float mx = -INFINITY;
-    for (int j = lane; j < nB; j += 32) {
-      const bool cand = !reduced || ((bits[j >> 5] >> (j & 31)) & 1u);
-      if (cand) mx = fmaxf(mx, srow[j]);
-    }
+    float* prow = prow_base + (size_t)r * nB;
+    for (int j0 = lane; j0 < nB; j0 += 32 * kU) {
+      float x[kU];
+      bool cand[kU];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-    for (int j = lane; j < nB; j += 32) {
-      const bool cand = !reduced || ((bits[j >> 5] >> (j & 31)) & 1u);
-      const float e = cand ? expf(srow[j] - mx) : 0.f;
-      srow[j] = e;
-      sum += e;
-    }
+      for (int u = 0; u < kU; ++u) {
+        const int j = j0 + 32 * u;
+        cand[u] = j < nB && !empty && (!reduced || ((bits[j >> 5] >> (j & 31)) & 1u));
+        x[u] = cand[u] ? prow[j] : 0.f;
+      }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    float* prow = probs + ((size_t)bh * nB + i0 + r) * nB;
-    const bool empty = !(mx > -INFINITY);
-    for (int j = lane; j < nB; j += 32) prow[j] = empty ? 0.f : srow[j] / sum;
+      for (int u = 0; u < kU; ++u) {
+        const int j = j0 + 32 * u;
+        if (j < nB) prow[j] = cand[u] ? expf(x[u] - ms.x) / ms.y : 0.f;
+      }
+    }
   }
 }
 
@@ -217,11 +304,11 @@ template <int D>
 static cudaError_t launch_scores_d(const float* qbar, const float* kbar, int BH, int nB,
                                    float scale, const int32_t* crp, const int32_t* cc,
                                    float* probs, unsigned* err, cudaStream_t s) {
-  const size_t smem = scores_smem_bytes(nB);
+  const size_t smem = ScoreSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  block_scores_kernel<D><<<dim3(ceil_div(nB, kRows), BH), 256, smem, s>>>(
+  block_scores_kernel<D><<<dim3(ceil_div(nB, kTile), BH), 256, smem, s>>>(
       qbar, kbar, nB, scale, crp, cc, probs, err);
   return cudaGetLastError();
 }

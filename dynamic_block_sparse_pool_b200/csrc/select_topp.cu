@@ -11,11 +11,12 @@
 // below 2^150, so sums of up to 1024 of them fit in 192 bits and every
 // summation order gives the same cut.
 //
-// Kernel 1 (select): one warp per row.  Keys (prob bits, inverted index) for
-//   up to 32 * R blocks sit in registers (R per lane) and are sorted by a
-//   bitonic network (in-register and shuffle compare-exchange); a warp scan
-//   of 192-bit lane sums finds the cut; the kept set becomes a 1024-bit mask
-//   plus a count.
+// Kernel 1 (select): one warp per row, no sort.  The kept set is every block
+//   above a threshold value tau plus, at tau itself, the first few ties in
+//   index order; tau comes from a bisection over the fp32 bit patterns with
+//   fp64 sums, accepted when the fp64 error bound decides the cut and
+//   otherwise settled with exact 192-bit sums.  The kept set becomes a
+//   1024-bit mask (one ballot per register) plus a count.
 // Kernel 2 (scan): exclusive scan of the counts into row_ptr (one CTA).
 // Kernel 3 (compact): one warp per row writes the kept indices ascending.
 #include <cstring>
@@ -70,63 +71,17 @@ __host__ __device__ __forceinline__ U192 fixed_of_bits(uint32_t bits) {
 
 constexpr unsigned FULL = 0xffffffffu;
 
-// Compare-exchange of the in-register pairs (r, r | J) of a bitonic stage;
-// positions are lane * R + r, and block size k decides the direction.
-template <int J, int R>
-__device__ __forceinline__ void bitonic_in_lane(uint64_t (&key)[R], int lane, int k) {
-  if constexpr (J < R) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if ((r & J) == 0) {
-        const int pr = r | J;
-        const bool desc = ((lane * R + r) & k) == 0;
-        const uint64_t a = key[r], b = key[pr];
-        const bool sw = desc ? (a < b) : (a > b);
-        key[r] = sw ? b : a;
-        key[pr] = sw ? a : b;
-      }
-    }
-  }
+// a * m for a small multiplier m (the result stays below 2^192 for the
+// values used here: a <= 2^149, m <= 1024).
+__device__ __forceinline__ U192 mul192(const U192& a, uint32_t m) {
+  const uint64_t p0 = a.w0 * m, c0 = __umul64hi(a.w0, m);
+  const uint64_t p1 = a.w1 * m, c1 = __umul64hi(a.w1, m);
+  U192 r;
+  r.w0 = p0;
+  r.w1 = p1 + c0;
+  r.w2 = a.w2 * m + c1 + (r.w1 < p1);
+  return r;
 }
-
-// Bitonic sort of 32 * R keys held R per lane, descending; afterwards lane L
-// holds sorted positions L*R .. L*R + R - 1.  The (k, j) stages are runtime
-// loops so the code stays small (a fully unrolled 1024-key network does not
-// fit the instruction cache); register indices stay compile-time constants.
-template <int R>
-__device__ __forceinline__ void bitonic_sort_desc(uint64_t (&key)[R], int lane) {
-#pragma unroll 1
-  for (int k = 2; k <= 32 * R; k <<= 1) {
-#pragma unroll 1
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j >= R) {
-        const int lm = j / R;
-        const bool lower = (lane & lm) == 0;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint64_t o = __shfl_xor_sync(FULL, key[r], lm);
-          const bool desc = ((lane * R + r) & k) == 0;
-          const bool take_max = lower == desc;
-          key[r] = take_max ? (key[r] > o ? key[r] : o) : (key[r] < o ? key[r] : o);
-        }
-      } else {
-        switch (j) {
-          case 16: bitonic_in_lane<16>(key, lane, k); break;
-          case 8: bitonic_in_lane<8>(key, lane, k); break;
-          case 4: bitonic_in_lane<4>(key, lane, k); break;
-          case 2: bitonic_in_lane<2>(key, lane, k); break;
-          default: bitonic_in_lane<1>(key, lane, k); break;
-        }
-      }
-    }
-  }
-}
-
-// Level of a probability for the threshold search: its exponent and the top
-// three mantissa bits (values within 12.5 % share a level).  Probabilities
-// are in [0, 1], so levels run from 0 to 1016.
-__device__ __forceinline__ int level_of(uint32_t bits) { return (int)(bits >> 20); }
-constexpr int kLevels = 1017;
 
 __device__ __forceinline__ U192 warp_sum192(U192 v) {
 #pragma unroll
@@ -140,110 +95,132 @@ __device__ __forceinline__ U192 warp_sum192(U192 v) {
   return v;
 }
 
-template <int R>
-__device__ __forceinline__ double level_sum_f64(const uint32_t (&bits)[R], uint32_t valid, int lv) {
-  double s = 0.0;
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-    if (((valid >> r) & 1u) && level_of(bits[r]) >= lv) s += (double)__uint_as_float(bits[r]);
+// Butterfly sum: every lane ends with the same value (fp addition is
+// commutative), so decisions taken on it are warp-uniform.
+__device__ __forceinline__ double warp_sum_f64(double s) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(FULL, s, off);
   return s;
 }
 
-// Sorts the n boundary keys of a warp (in shared memory) descending and
-// returns how many of them, taken in order, first bring the running exact
-// sum `base` to `target` (n if none does).  R = keys per lane.
-template <int R>
-__device__ __noinline__ int boundary_cut(uint64_t* keys, int n, U192 base, const U192 target,
-                                         int lane) {
-  uint64_t key[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int i = lane * R + r;
-    key[r] = i < n ? keys[i] : 0ull;
-  }
-  bitonic_sort_desc<R>(key, lane);
-  U192 own{0ull, 0ull, 0ull};
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-    if (key[r]) add192(own, fixed_of_bits((uint32_t)(key[r] >> 32) - 1u));
-  U192 incl = own;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    U192 o;
-    o.w0 = __shfl_up_sync(FULL, incl.w0, off);
-    o.w1 = __shfl_up_sync(FULL, incl.w1, off);
-    o.w2 = __shfl_up_sync(FULL, incl.w2, off);
-    if (lane >= off) add192(incl, o);
-  }
-  U192 excl;
-  excl.w0 = __shfl_up_sync(FULL, incl.w0, 1);
-  excl.w1 = __shfl_up_sync(FULL, incl.w1, 1);
-  excl.w2 = __shfl_up_sync(FULL, incl.w2, 1);
-  if (lane == 0) excl = U192{0ull, 0ull, 0ull};
-  U192 ti = incl;
-  add192(ti, base);
-  const unsigned ball = __ballot_sync(FULL, ge192(ti, target));
-  int cut = n;
-  if (ball) {
-    const int L = __ffs(ball) - 1;
-    int kk = 0;
-    if (lane == L) {
-      U192 acc = excl;
-      add192(acc, base);
-      bool done = false;
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (!done && key[r]) {
-          add192(acc, fixed_of_bits((uint32_t)(key[r] >> 32) - 1u));
-          if (ge192(acc, target)) {
-            kk = L * R + r + 1;
-            done = true;
-          }
-        }
-      }
-    }
-    cut = __shfl_sync(FULL, kk, L);
-  }
-  // write the sorted order back so the caller can mark the first `cut`
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int i = lane * R + r;
-    if (i < n) keys[i] = key[r];
-  }
-  __syncwarp();
-  return cut;
+__device__ __forceinline__ uint32_t key_of(double v) { return __float_as_uint((float)v); }
+
+// Candidate c * 32 + lane of a row, read from memory: its key (bit pattern
+// of the probability, sanitised like the main load) or false if it is not a
+// candidate.
+__device__ __forceinline__ bool load_key(const float* __restrict__ prow, const uint32_t* cbits,
+                                         int nB, int c, int lane, uint32_t& key) {
+  const int e = c * 32 + lane;
+  if (e >= nB || (cbits != nullptr && !((cbits[c] >> lane) & 1u))) return false;
+  const float f = prow[e];
+  key = (f >= 0.f && f <= 1.f) ? (__float_as_uint(f) & 0x7FFFFFFFu) : 0u;
+  return true;
 }
 
-// One warp per row: values of up to 32 * R candidate blocks, R per lane
-// (element e = r * 32 + lane).
-//   1. A binary search over levels, with fp64 sums (exact to ~1e-13), finds
-//      the level t where the mass of everything at or above t first reaches p.
-//   2. An exact 192-bit pass verifies mass(level > t) < p <= mass(level >= t)
-//      and moves t by one level if rounding misled the search.
-//   3. Everything above level t is kept.  The few blocks on level t are
-//      sorted by (probability desc, index asc) and kept until the exact sum
-//      reaches p.
+// Exact selection of one row with 192-bit sums, re-reading the row from
+// memory (used only when the fp64 search cannot decide: a prefix mass within
+// the fp64 error of p, or several blocks tied at the threshold).
+//   tau: starting guess for the threshold key (-1: keep everything).  Each
+//   correction moves it to the neighbouring key present in the row, so the
+//   loop ends.  Then: keys > tau are kept, and the tie of rank k (0-based,
+//   index order) at tau is kept iff mass(key > tau) + k * tau < p.
+// Returns the number kept; lane L receives word L of the row bitmap.
+__device__ __noinline__ int select_row_exact(const float* __restrict__ prow, const uint32_t* cbits,
+                                             int nB, U192 target, int tau, int lane,
+                                             uint32_t& myword) {
+  const int nC = (nB + 31) >> 5;
+  U192 above{0ull, 0ull, 0ull};
+  for (int guard = 0; guard <= 32 * nC + 1; ++guard) {
+    U192 a{0ull, 0ull, 0ull};
+    int ties = 0;
+    for (int c = 0; c < nC; ++c) {
+      uint32_t k;
+      if (load_key(prow, cbits, nB, c, lane, k)) {
+        if ((int)k > tau) add192(a, fixed_of_bits(k));
+        else if ((int)k == tau) ++ties;
+      }
+    }
+    above = warp_sum192(a);
+    if (ge192(above, target)) {  // tau too low: next larger key present
+      uint32_t nxt = 0xFFFFFFFFu;
+      for (int c = 0; c < nC; ++c) {
+        uint32_t k;
+        if (load_key(prow, cbits, nB, c, lane, k) && (int)k > tau) nxt = min(nxt, k);
+      }
+      tau = (int)__reduce_min_sync(FULL, nxt);
+      continue;
+    }
+    if (tau >= 0) {
+      ties = (int)__reduce_add_sync(FULL, (unsigned)ties);
+      U192 all = mul192(fixed_of_bits((uint32_t)tau), (uint32_t)ties);
+      add192(all, above);
+      if (!ge192(all, target)) {  // tau too high: next smaller key, or keep all
+        int prv = -1;
+        for (int c = 0; c < nC; ++c) {
+          uint32_t k;
+          if (load_key(prow, cbits, nB, c, lane, k) && (int)k < tau) prv = max(prv, (int)k);
+        }
+        tau = __reduce_max_sync(FULL, prv);
+        continue;
+      }
+    }
+    break;
+  }
+  const U192 unit = tau >= 0 ? fixed_of_bits((uint32_t)tau) : U192{0ull, 0ull, 0ull};
+  int kept = 0, run = 0;
+  myword = 0u;
+  for (int c = 0; c < nC; ++c) {
+    uint32_t k = 0u;
+    const bool v = load_key(prow, cbits, nB, c, lane, k);
+    const bool tie = v && tau >= 0 && (int)k == tau;
+    const unsigned tb = __ballot_sync(FULL, tie);
+    bool keep = v && (tau < 0 || (int)k > tau);
+    if (tie) {
+      U192 pre = mul192(unit, (uint32_t)(run + __popc(tb & ((1u << lane) - 1u))));
+      add192(pre, above);
+      keep = !ge192(pre, target);
+    }
+    run += __popc(tb);
+    const unsigned w = __ballot_sync(FULL, keep);
+    kept += __popc(w);
+    if (lane == c) myword = w;
+  }
+  return kept;
+}
+
+// One warp per row; element e = r * 32 + lane is held by lane `lane` in
+// register r (R = ceil(nB / 32) registers).
+//
+// With the blocks ordered by (probability desc, index asc), the kept prefix
+// is {prob > tau} followed by the first m blocks (in index order) whose
+// probability equals tau, where tau is the largest probability with
+// mass(prob >= tau) >= p.  Non-negative fp32 values order like their bit
+// patterns (keys).
+//   1. Bisection over keys with fp64 sums.  Each pass sums the blocks at or
+//      above the midpoint and also finds the smallest of them and the
+//      largest block below it, so the lower end always sits on a present
+//      value and the search stops once no present value lies strictly
+//      between the two ends (about 10 passes on attention-map rows, against
+//      ~27 for a plain bisection of the key range).
+//   2. The fp64 sums of at most n terms in [0, 1] are within n * 2^-53 * T
+//      of exact (T: the row total).  When mass(>= tau) - p and p -
+//      mass(> tau) both exceed twice that, and tau is held by one block, the
+//      cut is decided: keep prob >= tau.  Otherwise (rare) the row is
+//      decided exactly with 192-bit sums.
+// If the whole row's mass is below p, every candidate is kept.
 template <int R>
-__global__ void __launch_bounds__(128)
-select_kernel(const float* __restrict__ probs, int rows, int nB, int p_one,
+__global__ void __launch_bounds__(128, 4)
+select_kernel(const float* __restrict__ probs, int rows, int nB, float p,
               uint64_t t0, uint64_t t1, uint64_t t2,
               const int32_t* __restrict__ cand_row_ptr, const int32_t* __restrict__ cand_col,
               uint32_t* __restrict__ bitmaps, int32_t* __restrict__ counts, unsigned* err) {
   __shared__ uint32_t cbits_all[4][32];
-  __shared__ uint32_t sel_all[4][32];
-  __shared__ uint64_t bkeys_all[4][32 * R];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 4 + warp;
   if (row >= rows) return;  // whole warp leaves together
   uint32_t* cbits = cbits_all[warp];
-  uint32_t* sel = sel_all[warp];
-  uint64_t* bkeys = bkeys_all[warp];
   const bool reduced = cand_row_ptr != nullptr;
-  const U192 target{t0, t1, t2};
 
-  sel[lane] = 0u;
   if (reduced) {
     cbits[lane] = 0u;
     __syncwarp();
@@ -260,119 +237,112 @@ select_kernel(const float* __restrict__ probs, int rows, int nB, int p_one,
         atomicOr(&cbits[j >> 5], 1u << (j & 31));
       }
     }
+    __syncwarp();
   }
-  __syncwarp();
 
   const float* prow = probs + (size_t)row * nB;
-  uint32_t bits[R];
+  double dv[R];         // candidate probabilities (0 for non-candidates)
   uint32_t valid = 0u;  // bit r: element r * 32 + lane is a candidate
 #pragma unroll
   for (int r = 0; r < R; ++r) {
+    dv[r] = 0.0;
     const int e = r * 32 + lane;
-    bits[r] = 0u;
-    if (e < nB && (!reduced || ((cbits[e >> 5] >> (e & 31)) & 1u))) {
+    if (e < nB && (!reduced || ((cbits[r] >> lane) & 1u))) {
       float f = prow[e];
       if (!(f >= 0.f && f <= 1.f)) {
         flag_error(err, kErrProb);
         f = 0.f;
       }
-      bits[r] = __float_as_uint(f) & 0x7FFFFFFFu;
+      dv[r] = (double)__uint_as_float(__float_as_uint(f) & 0x7FFFFFFFu);  // -0 -> +0
       valid |= 1u << r;
     }
   }
 
-  int kstar_extra = 0;  // boundary blocks kept (only when cut inside a level)
-  int t_level = -1;     // keep everything with level > t_level (-1: keep all)
-  int n_bnd = 0;
-  if (!p_one) {
-    // 1. threshold level from fp64 sums: largest t with mass(level >= t) >= p
-    const double tgt = ldexp((double)t0, -149) + ldexp((double)t1, -85) + ldexp((double)t2, -21);
-    int lo = -1, hi = kLevels;  // invariant: mass(>= lo) >= p (lo = -1: all), mass(>= hi) < p
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (level_sum_f64<R>(bits, valid, mid) >= tgt) lo = mid;
-      else hi = mid;
-    }
-    // 2. exact check of mass(level > t) < p <= mass(level >= t); fix by a level
-    int t = lo;
-    // each correction moves t one level towards the exact answer, so the loop
-    // ends; fp64 sums of at most 1024 non-negative terms are off by ~1e-13,
-    // which moves t by at most one level in practice
-    for (int guard = 0; guard <= kLevels + 1; ++guard) {
-      U192 above{0ull, 0ull, 0ull}, at_or_above{0ull, 0ull, 0ull};
+  int mode = 0;  // 0: keep every candidate, 1: keep prob >= tau_d, 2: exact path
+  double tau_d = 0.0;
+  int tau_key = -1;
+  if (p < 1.f) {
+    const double pd = (double)p;
+    double s = 0.0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) s += dv[r];
+    const double T = warp_sum_f64(s);
+    const int nv = (int)__reduce_add_sync(FULL, (unsigned)__popc(valid));
+    const double eps = (double)(nv + 1) * T * 0x1p-52;  // twice the fp64 error bound
+    if (T < pd) {
+      mode = T + eps < pd ? 0 : 2;
+    } else {
+      double mn = 2.0, mx = -1.0;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         if ((valid >> r) & 1u) {
-          const int lv = level_of(bits[r]);
-          if (lv >= t) {
-            const U192 x = fixed_of_bits(bits[r]);
-            add192(at_or_above, x);
-            if (lv > t) add192(above, x);
-          }
+          mn = fmin(mn, dv[r]);
+          mx = fmax(mx, dv[r]);
         }
       }
-      above = warp_sum192(above);
-      at_or_above = warp_sum192(at_or_above);
-      if (t >= 0 && !ge192(at_or_above, target)) {
-        --t;  // the fp64 search stopped one level too high
-        continue;
-      }
-      if (ge192(above, target)) {
-        ++t;  // one level too low
-        continue;
-      }
-      // 3. blocks on level t, compacted in index order, then sorted and cut
-      if (t >= 0) {
-        int mine = 0;
 #pragma unroll
-        for (int r = 0; r < R; ++r)
-          if (((valid >> r) & 1u) && level_of(bits[r]) == t) ++mine;
-        int incl = mine;
+      for (int off = 16; off > 0; off >>= 1) {
+        mn = fmin(mn, __shfl_xor_sync(FULL, mn, off));
+        mx = fmax(mx, __shfl_xor_sync(FULL, mx, off));
+      }
+      // invariants: lo is a present value with G(lo) = g_lo >= p; G(hi) =
+      // g_hi < p; below_hi = the largest present value below hi
+      double lo = mn, below_hi = mx, g_lo = T, g_hi = 0.0;
+      uint32_t hi_key = key_of(mx) + 1u;
+      while (below_hi != lo) {
+        const uint32_t mid = (key_of(lo) + hi_key) >> 1;  // lo < mid < hi
+        const double thr = (double)__uint_as_float(mid);
+        double s0 = 0.0, s1 = 0.0, up = 2.0, dn = -1.0;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int o = __shfl_up_sync(FULL, incl, off);
-          if (lane >= off) incl += o;
+        for (int r = 0; r < R; ++r) {
+          const bool ge = dv[r] >= thr;
+          if (r & 1) s1 += ge ? dv[r] : 0.0;
+          else s0 += ge ? dv[r] : 0.0;
+          up = ge ? fmin(up, dv[r]) : up;
+          dn = ge ? dn : fmax(dn, dv[r]);
         }
-        n_bnd = __shfl_sync(FULL, incl, 31);
-        int pos = incl - mine;
+        double g = s0 + s1;
 #pragma unroll
-        for (int r = 0; r < R; ++r)
-          if (((valid >> r) & 1u) && level_of(bits[r]) == t)
-            bkeys[pos++] = ((uint64_t)(bits[r] + 1u) << 32) |
-                           (uint64_t)(0xFFFFFFFFu - (uint32_t)(r * 32 + lane));
-        __syncwarp();
-        const int rb = (n_bnd + 31) / 32;
-        if (rb <= 1) kstar_extra = boundary_cut<1>(bkeys, n_bnd, above, target, lane);
-        else if (rb <= 2) kstar_extra = boundary_cut<2 <= R ? 2 : R>(bkeys, n_bnd, above, target, lane);
-        else if (rb <= 4) kstar_extra = boundary_cut<4 <= R ? 4 : R>(bkeys, n_bnd, above, target, lane);
-        else if (rb <= 8) kstar_extra = boundary_cut<8 <= R ? 8 : R>(bkeys, n_bnd, above, target, lane);
-        else if (rb <= 16) kstar_extra = boundary_cut<16 <= R ? 16 : R>(bkeys, n_bnd, above, target, lane);
-        else kstar_extra = boundary_cut<R>(bkeys, n_bnd, above, target, lane);
+        for (int off = 16; off > 0; off >>= 1) {
+          g += __shfl_xor_sync(FULL, g, off);
+          up = fmin(up, __shfl_xor_sync(FULL, up, off));
+          dn = fmax(dn, __shfl_xor_sync(FULL, dn, off));
+        }
+        if (g >= pd) {
+          lo = up;
+          g_lo = g;
+        } else {
+          hi_key = mid;
+          g_hi = g;
+          below_hi = dn;
+        }
       }
-      t_level = t;
-      break;
+      int ties = 0;
+#pragma unroll
+      for (int r = 0; r < R; ++r) ties += (((valid >> r) & 1u) && dv[r] == lo) ? 1 : 0;
+      ties = (int)__reduce_add_sync(FULL, (unsigned)ties);
+      tau_d = lo;
+      tau_key = (int)key_of(lo);
+      mode = (g_lo - eps >= pd && g_hi + eps < pd && ties == 1) ? 1 : 2;
     }
   }
 
-  // keep: level > t_level, plus the first kstar_extra sorted boundary blocks
+  uint32_t myword = 0u;
   int kept = 0;
+  if (mode == 2) {
+    kept = select_row_exact(prow, reduced ? cbits : nullptr, nB, U192{t0, t1, t2}, tau_key, lane,
+                            myword);
+  } else {
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (((valid >> r) & 1u) && level_of(bits[r]) > t_level) {
-      const int e = r * 32 + lane;
-      atomicOr(&sel[e >> 5], 1u << (e & 31));
-      ++kept;
+    for (int r = 0; r < R; ++r) {
+      const bool keep = ((valid >> r) & 1u) && (mode == 0 || dv[r] >= tau_d);
+      const unsigned w = __ballot_sync(FULL, keep);
+      kept += __popc(w);
+      if (lane == r) myword = w;
     }
   }
-  for (int i = lane; i < kstar_extra; i += 32) {
-    const uint32_t e = 0xFFFFFFFFu - (uint32_t)bkeys[i];
-    atomicOr(&sel[e >> 5], 1u << (e & 31));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(FULL, kept, o);
-  __syncwarp();
-  bitmaps[(size_t)row * 32 + lane] = sel[lane];
-  if (lane == 0) counts[row] = kept + kstar_extra;
+  bitmaps[(size_t)row * 32 + lane] = myword;
+  if (lane == 0) counts[row] = kept;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -457,19 +427,24 @@ cudaError_t launch_select(const float* probs, int rows, int nB, float p,
                           int32_t* counts, unsigned* err, cudaStream_t s) {
   uint32_t pbits;
   memcpy(&pbits, &p, sizeof(pbits));
-  const int p_one = p >= 1.0f ? 1 : 0;
-  const U192 t = fixed_of_bits(p_one ? 0x3F800000u : pbits);
+  const U192 t = fixed_of_bits(p >= 1.0f ? 0x3F800000u : pbits);
   const int grid = ceil_div(rows, 8);
-  const int R = nB <= 32 ? 1 : nB <= 64 ? 2 : nB <= 128 ? 4 : nB <= 256 ? 8 : nB <= 512 ? 16 : 32;
+  const int R = ceil_div(nB, 32);  // registers per lane, 1 .. 32
   switch (R) {
 #define DSA_SEL(RR)                                                                            \
   case RR:                                                                                     \
-    select_kernel<RR><<<ceil_div(rows, 4), 128, 0, s>>>(probs, rows, nB, p_one, t.w0, t.w1,   \
-                                                        t.w2, cand_row_ptr, cand_col, bitmaps, \
+    select_kernel<RR><<<ceil_div(rows, 4), 128, 0, s>>>(probs, rows, nB, p, t.w0, t.w1, t.w2,  \
+                                                        cand_row_ptr, cand_col, bitmaps,       \
                                                         counts, err);                          \
     break;
-    DSA_SEL(1) DSA_SEL(2) DSA_SEL(4) DSA_SEL(8) DSA_SEL(16) DSA_SEL(32)
+    DSA_SEL(1) DSA_SEL(2) DSA_SEL(3) DSA_SEL(4) DSA_SEL(5) DSA_SEL(6) DSA_SEL(7) DSA_SEL(8)
+    DSA_SEL(9) DSA_SEL(10) DSA_SEL(11) DSA_SEL(12) DSA_SEL(13) DSA_SEL(14) DSA_SEL(15)
+    DSA_SEL(16) DSA_SEL(17) DSA_SEL(18) DSA_SEL(19) DSA_SEL(20) DSA_SEL(21) DSA_SEL(22)
+    DSA_SEL(23) DSA_SEL(24) DSA_SEL(25) DSA_SEL(26) DSA_SEL(27) DSA_SEL(28) DSA_SEL(29)
+    DSA_SEL(30) DSA_SEL(31) DSA_SEL(32)
 #undef DSA_SEL
+    default:
+      return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
