@@ -28,13 +28,15 @@
 // from one thread execute in order: S(it+3) overwrites buffer it % 3 only
 // after PV(it) has read P(it) from it.
 //
-// Online softmax with a lazy reference: the running max m_ref moves only when
-// a block's max exceeds it by more than 8 (log2 units); otherwise P is formed
-// against the stale reference (values up to 2^8, exact in fp32 and bf16), so
-// O is rarely rescaled.  A rescale of O at block it first waits until PV(it-1)
-// has finished.  O / l and lse use the same reference, so the result is
-// exact.  P is written back with the 16x128b layout, which puts each
-// thread's packed key pairs exactly where the MMA reads row-major P.
+// Online softmax with a lazy reference: the first block's row maxima set the
+// reference m_ref; later blocks form P = 2^(S*scale*log2e - m_ref) without
+// computing their maxima.  P up to 2^64 is harmless (bf16 and fp32 carry it
+// as precisely as small values), so only a block whose partial row sums
+// reach 2^64 (or overflow) is redone: its maxima become the new reference,
+// and O (after PV(it-1) has finished) and the running sums are rescaled.
+// O / l and lse use the same reference, so the result is exact.  P is
+// written back with the 16x128b layout, which puts each thread's packed key
+// pairs exactly where the MMA reads row-major P.
 //
 // Each selected block's log-sum (for the exact block mass) is
 // m_ref + log2(sum of that block's P row), written per query row.
@@ -60,7 +62,7 @@ constexpr int kSBufs = 3;       // S/P buffers in tensor memory
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 384;
 constexpr float kLn2 = 0.69314718055994530942f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kPMax = 0x1p64f;  // partial row sums at or above this redo the block
 
 // mbarrier slots
 enum : int {
@@ -96,26 +98,6 @@ __device__ __forceinline__ float exp2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe, for x <= 8 (softmax arguments here never exceed the
-// rescale threshold).  Cody-Waite style reduction x = n + f with n = round(x)
-// (the 1.5 * 2^23 rounding constant) and |f| <= 1/2, then a degree-4
-// polynomial for 2^f fitted for minimum maximum relative error on
-// [-1/2, 1/2] (Lawson's iteratively reweighted least squares; max relative
-// error 2.7e-6 when evaluated in fp32), then n is added to the exponent
-// field.  Arguments below -125 (including -inf) give 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.0f);
-  const float t = xc + 12582912.0f;
-  const float f = xc - (t - 12582912.0f);
-  float p = fmaf(0x1.3997d4p-7f, f, 0x1.ca1442p-5f);
-  p = fmaf(p, f, 0x1.ec06dap-3f);
-  p = fmaf(p, f, 0x1.62e0dcp-1f);
-  p = fmaf(p, f, 0x1.ffffe8p-1f);
-  const int n = __float_as_int(t) - 0x4B400000;
-  const float y = __int_as_float(__float_as_int(p) + (n << 23));
-  return x < -125.0f ? 0.0f : y;
 }
 
 template <int D>
@@ -323,7 +305,18 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     float mref_a = -INFINITY, mref_b = -INFINITY;  // reference maxima (log2 units)
     float l_a = 0.f, l_b = 0.f;                    // this thread's share of the row sums
     bool failed = false;
-    for (int it = 0; it < n; ++it) {
+    // Warps 4-7 start half a block behind warps 0-3 (they begin once S(1) is
+    // ready, one S MMA later than S(0)), so the two softmax warps of each SM
+    // sub-partition are out of phase: one is in its exp2 stretch (MUFU-bound)
+    // while the other loads, reduces and stores.  The lag is stable: S is
+    // triple-buffered and the leading warps never wait for the trailing ones
+    // except through PV(it) -> S(it + 3).  (S(4) cannot complete before these
+    // warps have produced P(1), so the wait below sees the first phase of
+    // buffer 1.)
+    if ((warp >> 2) == 1 && n > 1) {
+      if (!warp_all(mbar_wait(bar(kBarSFull + 1), 0u))) failed = true;
+    }
+    for (int it = 0; it < n && !failed; ++it) {
       const int b = it % kSBufs;
       const uint32_t tS = tmem + lane_off + 128u * (uint32_t)b;
       if (!warp_all(mbar_wait(bar(kBarSFull + b), (uint32_t)(it / kSBufs) & 1u)) ||
@@ -348,57 +341,78 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               sv[4 * k + 2 + u] = __float_as_uint(-INFINITY);
             }
       }
-      float ma4[4], mb4[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        ma4[u] = fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1]));
-        mb4[u] = fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]));
-      }
-#pragma unroll
-      for (int k = 4; k < 16; ++k) {
-        ma4[k & 3] = fmaxf(ma4[k & 3], fmaxf(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1])));
-        mb4[k & 3] = fmaxf(mb4[k & 3], fmaxf(__uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3])));
-      }
-      float ma = fmaxf(fmaxf(ma4[0], ma4[1]), fmaxf(ma4[2], ma4[3]));
-      float mb = fmaxf(fmaxf(mb4[0], mb4[1]), fmaxf(mb4[2], mb4[3]));
-      ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
-      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
-      ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
-      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-      const float xa = ma * scale_log2, xb = mb * scale_log2;
-      const bool need_a = xa > mref_a + kRescaleThreshold;
-      const bool need_b = xb > mref_b + kRescaleThreshold;
-      const bool warp_need = __any_sync(0xffffffffu, need_a || need_b);
-      float alpha_a = 1.0f, alpha_b = 1.0f;
-      if (need_a) {
-        alpha_a = exp2f(mref_a - xa);  // 0 on the first block
-        l_a *= alpha_a;
-        mref_a = xa;
-      }
-      if (need_b) {
-        alpha_b = exp2f(mref_b - xb);
-        l_b *= alpha_b;
-        mref_b = xb;
-      }
-      // P = 2^(S*scale*log2e - m_ref); pk[2k]: row ra, packed keys (8k+2t0, 8k+2t0+1),
-      // pk[2k+1]: row rb -- the 16x128b layout of packed column 4k + t0
-      float rsa[2] = {0.f, 0.f}, rsb[2] = {0.f, 0.f};
+      // The exps run against the reference; the row maxima are computed only
+      // for the first block, or when a thread's partial row sums show the
+      // reference has fallen far below this block's maxima.
+      const uint64_t sc2 = pack_f32x2(scale_log2, scale_log2);
       uint32_t pk[32];
+      float rs_a = 0.f, rs_b = 0.f;
+      auto exps = [&]() {
+        const uint64_t na2 = pack_f32x2(-mref_a, -mref_a), nb2 = pack_f32x2(-mref_b, -mref_b);
+        uint64_t rsa2[2] = {0ull, 0ull}, rsb2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float a0 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k]), scale_log2, -mref_a));
-        const float a1 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k + 1]), scale_log2, -mref_a));
-        const float b0 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k + 2]), scale_log2, -mref_b));
-        const float b1 = exp2_mufu(fmaf(__uint_as_float(sv[4 * k + 3]), scale_log2, -mref_b));
-        rsa[k & 1] += a0 + a1;
-        rsb[k & 1] += b0 + b1;
-        const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1);  // .x = lower key, low half
-        const __nv_bfloat162 hb = __floats2bfloat162_rn(b0, b1);
-        pk[2 * k] = *reinterpret_cast<const uint32_t*>(&ha);
-        pk[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&hb);
+        for (int k = 0; k < 16; ++k) {
+          float a0, a1, b0, b1;
+          unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1])), sc2, na2), a0, a1);
+          unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3])), sc2, nb2), b0, b1);
+          a0 = exp2_mufu(a0);
+          a1 = exp2_mufu(a1);
+          b0 = exp2_mufu(b0);
+          b1 = exp2_mufu(b1);
+          rsa2[k & 1] = add_f32x2(rsa2[k & 1], pack_f32x2(a0, a1));
+          rsb2[k & 1] = add_f32x2(rsb2[k & 1], pack_f32x2(b0, b1));
+          const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1);
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(b0, b1);
+          pk[2 * k] = *reinterpret_cast<const uint32_t*>(&ha);
+          pk[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&hb);
+        }
+        float u0, u1, u2, u3;
+        unpack_f32x2(add_f32x2(rsa2[0], rsa2[1]), u0, u1);
+        unpack_f32x2(add_f32x2(rsb2[0], rsb2[1]), u2, u3);
+        rs_a = u0 + u1;
+        rs_b = u2 + u3;
+      };
+      float alpha_a = 1.0f, alpha_b = 1.0f;
+      bool warp_need = false;
+      auto new_reference = [&]() {
+        float ma4[4], mb4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          ma4[u] = fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1]));
+          mb4[u] = fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]));
+        }
+#pragma unroll
+        for (int k = 4; k < 16; ++k) {
+          ma4[k & 3] = max3f(ma4[k & 3], __uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1]));
+          mb4[k & 3] = max3f(mb4[k & 3], __uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3]));
+        }
+        float ma = max3f(ma4[0], ma4[1], fmaxf(ma4[2], ma4[3]));
+        float mb = max3f(mb4[0], mb4[1], fmaxf(mb4[2], mb4[3]));
+        ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+        ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+        const float xa = ma * scale_log2, xb = mb * scale_log2;
+        const bool need_a = xa > mref_a, need_b = xb > mref_b;
+        warp_need = __any_sync(0xffffffffu, need_a || need_b);
+        if (need_a) {
+          alpha_a = exp2f(mref_a - xa);  // 0 on the first block
+          l_a *= alpha_a;
+          mref_a = xa;
+        }
+        if (need_b) {
+          alpha_b = exp2f(mref_b - xb);
+          l_b *= alpha_b;
+          mref_b = xb;
+        }
+      };
+      if (it == 0) new_reference();
+      exps();
+      if (it > 0 && __any_sync(0xffffffffu, !(rs_a < kPMax) || !(rs_b < kPMax))) {
+        new_reference();
+        exps();
       }
       tmem_st16x128b_x16(tS, pk);
-      const float rs_a = rsa[0] + rsa[1], rs_b = rsb[0] + rsb[1];
       if (warp_need && it > 0) {
         // O holds the sum through block it-1; wait for PV(it-1), then move O to
         // the new reference before PV(it) accumulates onto it

@@ -14,8 +14,8 @@
 // Kernel 1 (select): one warp per row, no sort.  The kept set is every block
 //   above a threshold value tau plus, at tau itself, the first few ties in
 //   index order; tau comes from a bisection over the fp32 bit patterns with
-//   fp64 sums, accepted when the fp64 error bound decides the cut and
-//   otherwise settled with exact 192-bit sums.  The kept set becomes a
+//   fp32 sums, accepted when an fp64 check with its error bound decides the
+//   cut and otherwise settled with exact 192-bit sums.  The kept set becomes a
 //   1024-bit mask (one ballot per register) plus a count.
 // Kernel 2 (scan): exclusive scan of the counts into row_ptr (one CTA).
 // Kernel 3 (compact): one warp per row writes the kept indices ascending.
@@ -103,8 +103,6 @@ __device__ __forceinline__ double warp_sum_f64(double s) {
   return s;
 }
 
-__device__ __forceinline__ uint32_t key_of(double v) { return __float_as_uint((float)v); }
-
 // Candidate c * 32 + lane of a row, read from memory: its key (bit pattern
 // of the probability, sanitised like the main load) or false if it is not a
 // candidate.
@@ -188,6 +186,12 @@ __device__ __noinline__ int select_row_exact(const float* __restrict__ prow, con
   return kept;
 }
 
+__device__ __forceinline__ float warp_sum_f32(float s) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(FULL, s, off);
+  return s;
+}
+
 // One warp per row; element e = r * 32 + lane is held by lane `lane` in
 // register r (R = ceil(nB / 32) registers).
 //
@@ -195,21 +199,23 @@ __device__ __noinline__ int select_row_exact(const float* __restrict__ prow, con
 // is {prob > tau} followed by the first m blocks (in index order) whose
 // probability equals tau, where tau is the largest probability with
 // mass(prob >= tau) >= p.  Non-negative fp32 values order like their bit
-// patterns (keys).
-//   1. Bisection over keys with fp64 sums.  Each pass sums the blocks at or
+// patterns (keys), so comparisons run on the integer keys.
+//   1. Bisection over keys with fp32 sums.  Each pass sums the blocks at or
 //      above the midpoint and also finds the smallest of them and the
 //      largest block below it, so the lower end always sits on a present
 //      value and the search stops once no present value lies strictly
 //      between the two ends (about 10 passes on attention-map rows, against
 //      ~27 for a plain bisection of the key range).
-//   2. The fp64 sums of at most n terms in [0, 1] are within n * 2^-53 * T
-//      of exact (T: the row total).  When mass(>= tau) - p and p -
-//      mass(> tau) both exceed twice that, and tau is held by one block, the
-//      cut is decided: keep prob >= tau.  Otherwise (rare) the row is
-//      decided exactly with 192-bit sums.
+//   2. One fp64 pass: mass(>= tau), mass(> tau), the number of blocks at
+//      tau and the row total T.  Sums of at most n terms in [0, 1] are
+//      within n * 2^-53 * T of exact; when mass(>= tau) - p and
+//      p - mass(> tau) both exceed twice that and tau is held by one block,
+//      the cut is decided: keep prob >= tau.  Otherwise (an fp32 search that
+//      went astray, a prefix mass within rounding of p, or ties at tau) the
+//      row is decided exactly with 192-bit sums.
 // If the whole row's mass is below p, every candidate is kept.
 template <int R>
-__global__ void __launch_bounds__(128, 4)
+__global__ void __launch_bounds__(128, 8)
 select_kernel(const float* __restrict__ probs, int rows, int nB, float p,
               uint64_t t0, uint64_t t1, uint64_t t2,
               const int32_t* __restrict__ cand_row_ptr, const int32_t* __restrict__ cand_col,
@@ -241,11 +247,11 @@ select_kernel(const float* __restrict__ probs, int rows, int nB, float p,
   }
 
   const float* prow = probs + (size_t)row * nB;
-  double dv[R];         // candidate probabilities (0 for non-candidates)
+  uint32_t kv[R];       // keys of the candidates (0 for non-candidates)
   uint32_t valid = 0u;  // bit r: element r * 32 + lane is a candidate
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    dv[r] = 0.0;
+    kv[r] = 0u;
     const int e = r * 32 + lane;
     if (e < nB && (!reduced || ((cbits[r] >> lane) & 1u))) {
       float f = prow[e];
@@ -253,89 +259,86 @@ select_kernel(const float* __restrict__ probs, int rows, int nB, float p,
         flag_error(err, kErrProb);
         f = 0.f;
       }
-      dv[r] = (double)__uint_as_float(__float_as_uint(f) & 0x7FFFFFFFu);  // -0 -> +0
+      kv[r] = __float_as_uint(f) & 0x7FFFFFFFu;  // -0 -> +0
       valid |= 1u << r;
     }
   }
 
-  int mode = 0;  // 0: keep every candidate, 1: keep prob >= tau_d, 2: exact path
-  double tau_d = 0.0;
-  int tau_key = -1;
+  int mode = 0;  // 0: keep every candidate, 1: keep key >= tau, 2: exact path
+  int tau = -1;
   if (p < 1.f) {
-    const double pd = (double)p;
-    double s = 0.0;
+    float s = 0.f;
 #pragma unroll
-    for (int r = 0; r < R; ++r) s += dv[r];
-    const double T = warp_sum_f64(s);
-    const int nv = (int)__reduce_add_sync(FULL, (unsigned)__popc(valid));
-    const double eps = (double)(nv + 1) * T * 0x1p-52;  // twice the fp64 error bound
-    if (T < pd) {
-      mode = T + eps < pd ? 0 : 2;
-    } else {
-      double mn = 2.0, mx = -1.0;
+    for (int r = 0; r < R; ++r) s += __uint_as_float(kv[r]);
+    if (warp_sum_f32(s) >= p) {
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         if ((valid >> r) & 1u) {
-          mn = fmin(mn, dv[r]);
-          mx = fmax(mx, dv[r]);
+          kmin = min(kmin, kv[r]);
+          kmax = max(kmax, kv[r]);
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        mn = fmin(mn, __shfl_xor_sync(FULL, mn, off));
-        mx = fmax(mx, __shfl_xor_sync(FULL, mx, off));
-      }
-      // invariants: lo is a present value with G(lo) = g_lo >= p; G(hi) =
-      // g_hi < p; below_hi = the largest present value below hi
-      double lo = mn, below_hi = mx, g_lo = T, g_hi = 0.0;
-      uint32_t hi_key = key_of(mx) + 1u;
+      // invariants: lo is a present key with G(lo) >= p; G(hi) < p;
+      // below_hi = the largest present key below hi
+      uint32_t lo = __reduce_min_sync(FULL, kmin);
+      uint32_t below_hi = __reduce_max_sync(FULL, kmax);
+      uint32_t hi = below_hi + 1u;
       while (below_hi != lo) {
-        const uint32_t mid = (key_of(lo) + hi_key) >> 1;  // lo < mid < hi
-        const double thr = (double)__uint_as_float(mid);
-        double s0 = 0.0, s1 = 0.0, up = 2.0, dn = -1.0;
+        const uint32_t mid = (lo + hi) >> 1;  // lo < mid < hi
+        float s0 = 0.f, s1 = 0.f;
+        uint32_t up = 0xFFFFFFFFu, dn = 0u;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const bool ge = dv[r] >= thr;
-          if (r & 1) s1 += ge ? dv[r] : 0.0;
-          else s0 += ge ? dv[r] : 0.0;
-          up = ge ? fmin(up, dv[r]) : up;
-          dn = ge ? dn : fmax(dn, dv[r]);
+          const bool ge = kv[r] >= mid;
+          if (r & 1) s1 += ge ? __uint_as_float(kv[r]) : 0.f;
+          else s0 += ge ? __uint_as_float(kv[r]) : 0.f;
+          up = min(up, ge ? kv[r] : 0xFFFFFFFFu);
+          dn = max(dn, ge ? 0u : kv[r]);
         }
-        double g = s0 + s1;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          g += __shfl_xor_sync(FULL, g, off);
-          up = fmin(up, __shfl_xor_sync(FULL, up, off));
-          dn = fmax(dn, __shfl_xor_sync(FULL, dn, off));
-        }
-        if (g >= pd) {
+        const float g = warp_sum_f32(s0 + s1);
+        up = __reduce_min_sync(FULL, up);
+        dn = __reduce_max_sync(FULL, dn);
+        if (g >= p) {
           lo = up;
-          g_lo = g;
         } else {
-          hi_key = mid;
-          g_hi = g;
+          hi = mid;
           below_hi = dn;
         }
       }
-      int ties = 0;
-#pragma unroll
-      for (int r = 0; r < R; ++r) ties += (((valid >> r) & 1u) && dv[r] == lo) ? 1 : 0;
-      ties = (int)__reduce_add_sync(FULL, (unsigned)ties);
-      tau_d = lo;
-      tau_key = (int)key_of(lo);
-      mode = (g_lo - eps >= pd && g_hi + eps < pd && ties == 1) ? 1 : 2;
+      tau = (int)lo;
     }
+    // 2. fp64 check of the cut
+    double g_ge = 0.0, g_gt = 0.0, tot = 0.0;
+    int ties = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const double d = (double)__uint_as_float(kv[r]);
+      tot += d;
+      if ((int)kv[r] >= tau) g_ge += d;
+      if ((int)kv[r] > tau) g_gt += d;
+      ties += (((valid >> r) & 1u) && (int)kv[r] == tau) ? 1 : 0;
+    }
+    tot = warp_sum_f64(tot);
+    g_ge = warp_sum_f64(g_ge);
+    g_gt = warp_sum_f64(g_gt);
+    ties = (int)__reduce_add_sync(FULL, (unsigned)ties);
+    const int nv = (int)__reduce_add_sync(FULL, (unsigned)__popc(valid));
+    const double pd = (double)p;
+    const double eps = (double)(nv + 1) * tot * 0x1p-52;  // twice the fp64 error bound
+    if (tau < 0) mode = tot + eps < pd ? 0 : 2;
+    else mode = (g_ge - eps >= pd && g_gt + eps < pd && ties == 1) ? 1 : 2;
   }
 
   uint32_t myword = 0u;
   int kept = 0;
   if (mode == 2) {
-    kept = select_row_exact(prow, reduced ? cbits : nullptr, nB, U192{t0, t1, t2}, tau_key, lane,
+    kept = select_row_exact(prow, reduced ? cbits : nullptr, nB, U192{t0, t1, t2}, tau, lane,
                             myword);
   } else {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const bool keep = ((valid >> r) & 1u) && (mode == 0 || dv[r] >= tau_d);
+      const bool keep = ((valid >> r) & 1u) && (mode == 0 || (int)kv[r] >= tau);
       const unsigned w = __ballot_sync(FULL, keep);
       kept += __popc(w);
       if (lane == r) myword = w;
