@@ -45,6 +45,8 @@
 // columns of D over the tensor {D, N, B*H}: rows past N are zero-filled and
 // masked to -inf.  No multicast.  Every mbarrier wait is bounded; a timeout
 // sets the device error word and the CTA winds down.
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace dsa {
@@ -64,18 +66,21 @@ constexpr uint32_t kTmemO = 384;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kPMax = 0x1p64f;  // partial row sums at or above this redo the block
 
-// mbarrier slots
+// mbarrier slots, one per ring stage (block it uses stage it % 3 of the K
+// and V rings and S buffer it % 3, so one barrier per event serves both the
+// ring and the buffer).  Each tcgen05.commit and each fence costs the tensor
+// pipe a few dozen cycles, so a block signals only two events:
+//   SFull:  S(it) is done -- S is ready for the softmax and K slot is free
+//   PVDone: PV(it) is done -- V slot is free, O holds blocks 0..it
+static_assert(kStages == kSBufs, "ring stages and S buffers share barriers");
 enum : int {
   kBarQ = 0,
-  kBarKFull = 1,                        // + stage
-  kBarKEmpty = kBarKFull + kStages,     // + stage
-  kBarVFull = kBarKEmpty + kStages,     // + stage
-  kBarVEmpty = kBarVFull + kStages,     // + stage
-  kBarSFull = kBarVEmpty + kStages,     // + S buffer
-  kBarPFull = kBarSFull + kSBufs,       // + S buffer (256 arrivals)
-  kBarPVDone = kBarPFull + kSBufs,      // + (block & 1)
-  kBarOFull = kBarPVDone + 2,
-  kNumBars = kBarOFull + 1
+  kBarKFull = 1,                        // + stage: K tile landed
+  kBarVFull = kBarKFull + kStages,      // + stage: V tile landed
+  kBarSFull = kBarVFull + kStages,      // + stage: S(it) done
+  kBarPFull = kBarSFull + kStages,      // + stage: P(it) written (one arrival per softmax warp)
+  kBarPVDone = kBarPFull + kStages,     // + stage: PV(it) done
+  kNumBars = kBarPVDone + kStages
 };
 
 template <int D>
@@ -92,6 +97,14 @@ struct SmemLayout {
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// log2(x) on the multi-function unit (the PTX approximate base-2 logarithm;
+// one instruction, absolute error ~1e-7 for the row sums it is used on).
+__device__ __forceinline__ float lg2_mufu(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // 2^x on the multi-function unit (the PTX approximate base-2 exponential).
 __device__ __forceinline__ float exp2_mufu(float x) {
@@ -146,7 +159,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp == kMmaWarp) {
     if (lane == 0) {
       for (int i = 0; i < kNumBars; ++i)
-        mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kSBufs) ? kSoftmaxThreads : 1);
+        mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kStages) ? kSoftmaxThreads / 32 : 1);
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -196,7 +209,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (step < n) {
           const int it = step, s = it % kStages;
           const int j = col_idx[s0 + it];
-          ok = mbar_wait(bar(kBarKEmpty + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
+          // K slot s is free once S(it - 3) is done
+          ok = mbar_wait(bar(kBarSFull + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
           if (!ok) break;
           mbar_expect_tx(bar(kBarKFull + s), kTileBytes);
           tma_tile<D>(sK + s * kTileBytes, &tmK, j * BN, bh, bar(kBarKFull + s));
@@ -205,7 +219,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (step >= kKLead) {
           const int it = step - kKLead, s = it % kStages;
           const int j = col_idx[s0 + it];
-          ok = mbar_wait(bar(kBarVEmpty + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
+          // V slot s is free once PV(it - 3) is done
+          ok = mbar_wait(bar(kBarPVDone + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
           if (!ok) break;
           mbar_expect_tx(bar(kBarVFull + s), kTileBytes);
           tma_tile<D>(sV + s * kTileBytes, &tmV, j * BN, bh, bar(kBarVFull + s));
@@ -225,73 +240,74 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issuer
-    if (lane == 0 && n > 0) {
-      // Every shared-memory descriptor is formed once here: the issuing
-      // thread shares its SM sub-partition with two busy softmax warps, so
-      // each MMA should cost it as few instructions as possible.
-      uint64_t dq[D / 16], dk[kStages][D / 16], dv[kStages][BN / 16];
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
-        dq[kk] = smem_desc_sw128(sQ + off, 16, 1024);
-#pragma unroll
-        for (int st = 0; st < kStages; ++st)
-          dk[st][kk] = smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024);
-      }
-#pragma unroll
-      for (int st = 0; st < kStages; ++st)
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          dv[st][kk] = smem_desc_sw128(sV + st * kTileBytes + kk * 2048, L::kSub, 1024);
-      bool ok = mbar_wait(bar(kBarQ), 0u);
-      // S(it) = Q K^T into buffer it % 3; the ring stage is dispatched to
-      // compile-time indices so the descriptors stay in registers
-      auto s_mmas = [&](uint32_t d, const uint64_t (&k)[D / 16]) {
-        mma_ss(d, dq[0], k[0], kIdescS, 0u);
-#pragma unroll
-        for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, dq[kk], k[kk], kIdescS);
+    // The whole warp runs the loop, so the waits, descriptors and addresses
+    // stay warp-uniform; lane 0 issues each MMA and commit.  The issuing warp
+    // shares its SM sub-partition with two busy softmax warps, so every
+    // instruction it saves shortens the tensor pipe's gaps.  The block loop
+    // is unrolled by the ring depth, which makes every stage index and
+    // descriptor offset a compile-time constant.
+    if (n > 0) {
+      const bool leader = lane == 0;
+      // three base descriptors; every other one differs only in its start
+      // address field (address >> 4, 14 bits, no carry below 256 KB)
+      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sK, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sV, L::kSub, 1024);
+      auto kdesc = [](int kk) -> uint64_t {  // K step kk of a K-major tile
+        return (uint64_t)(((kk >> 2) * L::kSub + (kk & 3) * 32) >> 4);
       };
-      auto issue_s = [&](int it) {
-        const int s = it % kStages;
-        if (!(ok = ok && mbar_wait(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u))) return;
-        tc_fence_after();
-        const uint32_t d = tmem + 128u * (uint32_t)(it % kSBufs);
-        switch (s) {
-          case 0: s_mmas(d, dk[0]); break;
-          case 1: s_mmas(d, dk[1]); break;
-          default: s_mmas(d, dk[2]); break;
+      bool ok = warp_all(mbar_wait(bar(kBarQ), 0u));
+      // S(it) = Q K^T into buffer it % 3.  The TMA load and the MMA both act
+      // in the async proxy and are ordered by the mbarrier alone.
+      auto issue_s = [&](int it, auto stage) {
+        constexpr int s = decltype(stage)::value;
+        if (!(ok = ok && warp_all(mbar_wait(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u))))
+          return;
+        if (leader) {
+          const uint32_t d = tmem + 128u * s;
+          const uint64_t k0 = dk0 + (uint64_t)((s * kTileBytes) >> 4);
+          mma_ss(d, dq0 + kdesc(0), k0 + kdesc(0), kIdescS, 0u);
+#pragma unroll
+          for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, dq0 + kdesc(kk), k0 + kdesc(kk), kIdescS);
+          mma_commit(bar(kBarSFull + s));
         }
-        mma_commit(bar(kBarKEmpty + s));
-        mma_commit(bar(kBarSFull + it % kSBufs));
+        __syncwarp();
       };
-      // O += P(it) V(it), P from tensor memory
-      auto pv_mmas = [&](uint32_t p, bool first, const uint64_t (&v)[BN / 16]) {
-        if (first)
-          mma_ts(tmem + kTmemO, p, v[0], kIdescO, 0u);
-        else
-          mma_ts_acc(tmem + kTmemO, p, v[0], kIdescO);
-#pragma unroll
-        for (int kk = 1; kk < BN / 16; ++kk) mma_ts_acc(tmem + kTmemO, p + kk * 8, v[kk], kIdescO);
-      };
-      for (int it = 0; it < n && it < kSBufs; ++it) issue_s(it);
-      for (int it = 0; it < n && ok && !*abort_flag; ++it) {
-        const int b = it % kSBufs, s = it % kStages;
-        const uint32_t ph = (uint32_t)(it / kSBufs) & 1u;
-        if (!(ok = mbar_wait(bar(kBarPFull + b), ph))) break;
-        if (!(ok = mbar_wait(bar(kBarVFull + s), (uint32_t)(it / kStages) & 1u))) break;
+      // O += P(it) V(it), P from tensor memory; then S(it + 3) into the same buffer
+      auto block = [&](int it, auto stage) {
+        constexpr int s = decltype(stage)::value;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (!(ok = ok && warp_all(mbar_wait(bar(kBarPFull + s), ph)) &&
+                   warp_all(mbar_wait(bar(kBarVFull + s), ph))))
+          return;
         tc_fence_after();
-        const uint32_t p = tmem + 128u * (uint32_t)b;
-        switch (s) {
-          case 0: pv_mmas(p, it == 0, dv[0]); break;
-          case 1: pv_mmas(p, it == 0, dv[1]); break;
-          default: pv_mmas(p, it == 0, dv[2]); break;
+        if (leader) {
+          const uint32_t p = tmem + 128u * s;
+          const uint64_t v0 = dv0 + (uint64_t)((s * kTileBytes) >> 4);
+          if (it == 0)
+            mma_ts(tmem + kTmemO, p, v0, kIdescO, 0u);
+          else
+            mma_ts_acc(tmem + kTmemO, p, v0, kIdescO);
+#pragma unroll
+          for (int kk = 1; kk < BN / 16; ++kk)
+            mma_ts_acc(tmem + kTmemO, p + kk * 8, v0 + (uint64_t)((kk * 2048) >> 4), kIdescO);
+          mma_commit(bar(kBarPVDone + s));
         }
-        mma_commit(bar(kBarVEmpty + s));
-        mma_commit(bar(kBarPVDone + (it & 1)));
-        if (it == n - 1) mma_commit(bar(kBarOFull));
-        if (it + kSBufs < n) issue_s(it + kSBufs);
+        __syncwarp();
+        if (it + kStages < n) issue_s(it + kStages, stage);
+      };
+      using S0 = std::integral_constant<int, 0>;
+      using S1 = std::integral_constant<int, 1>;
+      using S2 = std::integral_constant<int, 2>;
+      issue_s(0, S0{});
+      if (n > 1) issue_s(1, S1{});
+      if (n > 2) issue_s(2, S2{});
+      for (int it = 0; it < n && ok; it += kStages) {
+        block(it, S0{});
+        if (it + 1 < n) block(it + 1, S1{});
+        if (it + 2 < n) block(it + 2, S2{});
       }
-      if (!ok) {
+      if (!ok && leader) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
       }
@@ -319,8 +335,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     for (int it = 0; it < n && !failed; ++it) {
       const int b = it % kSBufs;
       const uint32_t tS = tmem + lane_off + 128u * (uint32_t)b;
-      if (!warp_all(mbar_wait(bar(kBarSFull + b), (uint32_t)(it / kSBufs) & 1u)) ||
-          warp_all(*abort_flag != 0)) {
+      if (!warp_all(mbar_wait(bar(kBarSFull + b), (uint32_t)(it / kSBufs) & 1u))) {
         failed = true;
         break;
       }
@@ -416,8 +431,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (warp_need && it > 0) {
         // O holds the sum through block it-1; wait for PV(it-1), then move O to
         // the new reference before PV(it) accumulates onto it
-        const int pb = (it - 1) & 1;
-        if (!warp_all(mbar_wait(bar(kBarPVDone + pb), (uint32_t)((it - 1) >> 1) & 1u))) {
+        const int pb = (it - 1) % kStages;
+        if (!warp_all(mbar_wait(bar(kBarPVDone + pb), (uint32_t)((it - 1) / kStages) & 1u))) {
           *abort_flag = 1;
         } else {
           tc_fence_after();
@@ -442,7 +457,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       l_b += rs_b;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + b));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarPFull + b));
       if (blk_lse != nullptr) {
         // the block's share of each row's denominator: sum over the quad
         float ta = rs_a + __shfl_xor_sync(0xffffffffu, rs_a, 1);
@@ -450,8 +466,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         ta += __shfl_xor_sync(0xffffffffu, ta, 2);
         tb += __shfl_xor_sync(0xffffffffu, tb, 2);
         if (t0 == 0) {
-          if (ra < qlen) blk_lse[(size_t)(s0 + it) * BN + ra] = (mref_a + log2f(ta)) * kLn2;
-          if (rb < qlen) blk_lse[(size_t)(s0 + it) * BN + rb] = (mref_b + log2f(tb)) * kLn2;
+          if (ra < qlen) blk_lse[(size_t)(s0 + it) * BN + ra] = (mref_a + lg2_mufu(ta)) * kLn2;
+          if (rb < qlen) blk_lse[(size_t)(s0 + it) * BN + rb] = (mref_b + lg2_mufu(tb)) * kLn2;
         }
       }
     }
@@ -464,7 +480,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
       l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
       l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-      if (!warp_all(mbar_wait(bar(kBarOFull), 0u))) {
+      if (!warp_all(mbar_wait(bar(kBarPVDone + (n - 1) % kStages), (uint32_t)((n - 1) / kStages) & 1u))) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
       } else {
