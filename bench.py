@@ -308,6 +308,10 @@ def sweep(args):
         torch.cuda.synchronize(dev)
         return sum(a.elapsed_time(b) for a, b in ev) / reps
 
+    def steady(fn, est_ms, seconds=0.6):
+        reps = max(3, int(seconds * 1e3 / max(est_ms, 1e-2)))
+        return timed(lambda: [fn() for _ in range(reps)], 1) / reps
+
     def point(w, q, k, v, p, cand=None, dense=None, label=None, extra=None):
         B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
         nB, rows = w.n_blocks, w.BH * w.n_blocks
@@ -334,14 +338,17 @@ def sweep(args):
         t_m = timed(mass, reps)
         step = t_s + t_a + t_m
         if dense is not None:
-            # the whole step and the dense p = 1 reference, timed alternately so
-            # that both run at the same clocks (the part is power-capped)
-            sp, de = [], []
-            for _ in range(3):
-                # five steps queued back to back: the host stays ahead of the GPU
-                sp.append(timed(lambda: [(search(), attend(), mass()) for _ in range(5)], 1) / 5)
-                de.append(timed(dense, 1))
-            step_alt, dense_ms = sorted(sp)[1], sorted(de)[1]
+            # The whole step and the dense p = 1 reference (the same kernel
+            # over an all-blocks CSR, with the same outputs), each timed in
+            # steady state -- about 0.6 s of back-to-back work, queued ahead
+            # -- in two alternating rounds; the second round is kept.  The
+            # part is power-capped, so a short burst after a long kernel (or
+            # the other way round) would see different clocks.
+            step_fn = lambda: (search(), attend(), mass())
+            d_est = timed(dense, 1)
+            for _ in range(2):
+                step_alt = steady(step_fn, step)
+                dense_ms = steady(dense, d_est)
         line = {"sweep": label or w.name, "p": p, "reduced_search": cand is not None,
                 "density": nnz / (rows * nB), "executed_tflop": flops / 1e12,
                 "search_ms": t_s, "attn_ms": t_a, "mass_ms": t_m, "step_ms": step,
@@ -349,7 +356,7 @@ def sweep(args):
                 "step_tflops": flops / (step * 1e-3) / 1e12}
         if dense is not None:
             red = (4 * D * B * H * N * N) / flops
-            line.update({"dense_attn_ms": dense_ms, "step_ms_alternating": step_alt,
+            line.update({"dense_attn_ms": dense_ms, "step_ms_steady": step_alt,
                          "flop_reduction": red, "speedup_attn": dense_ms / t_a,
                          "speedup_pipeline": dense_ms / step_alt,
                          "pipeline_over_reduction": dense_ms / step_alt / red})
@@ -364,8 +371,10 @@ def sweep(args):
         rpa = (torch.arange(rows + 1, device=dev, dtype=torch.int64) * nB).to(torch.int32)
         cia = torch.arange(nB, device=dev, dtype=torch.int32).repeat(rows)
         out = torch.empty_like(q)
+        lse = torch.empty(B, H, N, device=dev)
+        bl = torch.empty(rows * nB, blk, device=dev)
         f = lambda: ops.attn_fwd(q, k, v, rpa, cia, blk, 1.0 / math.sqrt(D), out=out,
-                                 want_lse=False, want_blk_lse=False)
+                                 lse=lse, blk_lse=bl)
         f(); torch.cuda.synchronize(dev)
         return f
 
