@@ -404,6 +404,58 @@ def sweep(args):
     w = synth.COGVIDEOX
     q, k, v = synth.make_qkv(w, 0, device="cuda")
     point(w, q, k, v, 0.9, dense=dense_of(w, q, k, v))
+    del q, k, v
+    torch.cuda.empty_cache()
+    gsrs_run(timed)
+
+
+def gsrs_run(timed):
+    """The step policy (warm-up, searches on exact block masses, mask reuse)
+    over the HunyuanVideo-like 10-step inputs, against full attention at
+    every step; each whole run timed twice, alternating, the second kept."""
+    from dynamic_block_sparse_pool_b200.schedule import GsrsPolicy, GsrsRunner
+    dev = torch.device("cuda", 0)
+    w = synth.HUNYUAN
+    B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+    nB, rows = w.n_blocks, w.BH * w.n_blocks
+    pol = GsrsPolicy(10, 1, (0.95, 0.9, 0.85, 0.8))
+    inputs = [synth.make_qkv(w, seed, bandwidth=bw, device="cuda")
+              for _, _, bw, seed in synth.hunyuan_schedule(10)]
+    run = GsrsRunner(pol, B, H, N, D, blk, w.dtype, device=dev)
+    all_rp, all_col = run.all_rp, run.all_col
+    out = torch.empty_like(inputs[0][0])
+    scale = 1.0 / math.sqrt(D)
+
+    def sparse_run():
+        run.have_base, run.cur = False, None
+        for s, (q, k, v) in enumerate(inputs):
+            run.step(s, q, k, v)
+
+    def dense_run():
+        for q, k, v in inputs:
+            ops.attn_fwd(q, k, v, all_rp, all_col, blk, scale, out=out, want_lse=False,
+                         want_blk_lse=False)
+
+    # executed FLOPs: each step over the mask it attends to
+    run.have_base, run.cur = False, None
+    flops = 0
+    for s, (q, k, v) in enumerate(inputs):
+        res = run.step(s, q, k, v)
+        flops += executed_flops(res.mask[0], res.mask[1], N, blk, D, nB)[0]
+    ops.device_status(dev)
+    dense_flops = 10 * 4 * D * B * H * N * N
+    for _ in range(2):
+        t_sparse = timed(sparse_run, 1)
+        t_dense = timed(dense_run, 1)
+    red = dense_flops / flops
+    line = {"sweep": "step policy on hunyuanvideo-like 10-step inputs", "warmup": pol.warmup,
+            "p": list(pol.p), "search_steps": pol.searches(),
+            "kinds": [k for k, _ in pol.kinds()], "run_ms": t_sparse, "dense_run_ms": t_dense,
+            "executed_tflop": flops / 1e12, "dense_tflop": dense_flops / 1e12,
+            "speedup": t_dense / t_sparse, "flop_reduction": red,
+            "speedup_over_reduction": t_dense / t_sparse / red,
+            "run_tflops": flops / (t_sparse * 1e-3) / 1e12}
+    print(json.dumps(line), flush=True)
 
 # ---------------------------------------------------------------- GPU bench --
 

@@ -10,6 +10,11 @@
 // the attention kernel).  One CTA per CSR row; each of its 8 warps keeps the
 // row's lse values in registers and reduces every 8th slot, reading that
 // slot's block-size run of blk_lse once, coalesced.
+//
+// mass_to_probs scatters those masses back into dense rows, so that a Top-p
+// selection can run on exact attention weights (GSRS abstract: Top-p
+// selection supported by exact attention weights from the FlashAttention
+// pass; Figure 4: later searches evaluate only the candidate mask).
 #include "common.cuh"
 
 namespace dsa {
@@ -49,7 +54,45 @@ block_mass_kernel(const float* __restrict__ lse, const float* __restrict__ blk, 
   }
 }
 
+// Dense probability rows from the exact masses of a CSR mask: row r of
+// probs gets mass[s] at column col_idx[s] for each of its slots s and 0
+// elsewhere.  One warp per row: it zeroes the row (coalesced), then writes
+// its slots; __syncwarp orders the two.
+__global__ void __launch_bounds__(256)
+mass_to_probs_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                     const float* __restrict__ mass, int rows, int nB, float* __restrict__ probs,
+                     unsigned* err) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= rows) return;  // whole warp leaves together
+  float* prow = probs + (size_t)r * nB;
+  for (int j = lane; j < nB; j += 32) prow[j] = 0.f;
+  __syncwarp();
+  const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
+  if (s0 < 0 || s1 < s0) {
+    if (lane == 0) flag_error(err, kErrRowPtr);
+    return;
+  }
+  for (int s = s0 + lane; s < s1; s += 32) {
+    const int j = col_idx[s];
+    if (j < 0 || j >= nB) {
+      flag_error(err, kErrCsrIndex);
+      continue;
+    }
+    prow[j] = mass[s];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx,
+                                 const float* mass, int rows, int nB, float* probs,
+                                 unsigned* err, cudaStream_t s) {
+  if (rows > 0)
+    mass_to_probs_kernel<<<ceil_div(rows, 8), 256, 0, s>>>(row_ptr, col_idx, mass, rows, nB,
+                                                           probs, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,

@@ -56,6 +56,9 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int B
                               const int32_t* col_idx, void* out, float* lse,
                               float* blk_lse, unsigned* err, cudaStream_t s,
                               const char** why);
+cudaError_t launch_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx,
+                                 const float* mass, int rows, int nB, float* probs,
+                                 unsigned* err, cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

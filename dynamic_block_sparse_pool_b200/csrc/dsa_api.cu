@@ -221,6 +221,24 @@ dsa_status dsa_block_mass(const float* lse, const float* blk_lse, int B, int H, 
   return DSA_OK;
 }
 
+dsa_status dsa_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx, const float* mass,
+                             int rows, int nB, float* probs, void* stream) {
+  g_last_error.clear();
+  if (!row_ptr || !col_idx || !mass || !probs)
+    return fail(DSA_ERR_INVALID_ARG, "null row_ptr, col_idx, mass or probs");
+  if (rows < 1) return fail(DSA_ERR_INVALID_ARG, "rows must be >= 1 (got %d)", rows);
+  dsa_status st = check_blocks_limit(rows, nB);
+  if (st != DSA_OK) return st;
+  if (!aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(mass, 4) || !aligned(probs, 4))
+    return fail(DSA_ERR_INVALID_ARG, "misaligned pointer");
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  cudaError_t e = dsa::launch_mass_to_probs(row_ptr, col_idx, mass, rows, nB, probs, dev->err_word,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mass_to_probs launch");
+  return DSA_OK;
+}
+
 dsa_status dsa_device_status(void* stream) {
   g_last_error.clear();
   DeviceInfo* dev = nullptr;

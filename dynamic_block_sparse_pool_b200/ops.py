@@ -148,6 +148,21 @@ def block_mass(lse: torch.Tensor, blk_lse: torch.Tensor, row_ptr: torch.Tensor, 
     return mass
 
 
+def mass_to_probs(row_ptr: torch.Tensor, col_idx: torch.Tensor, mass: torch.Tensor, nB: int,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """probs [rows, nB] fp32: each row's exact block masses at their columns, 0 elsewhere."""
+    rows = row_ptr.numel() - 1
+    _check_csr((row_ptr, col_idx), rows)
+    if mass.dtype != torch.float32 or not mass.is_cuda:
+        raise ValueError("mass must be an fp32 CUDA tensor")
+    if out is None:
+        out = torch.empty(rows, nB, device=mass.device, dtype=torch.float32)
+    st = lib().dsa_mass_to_probs(row_ptr.data_ptr(), col_idx.data_ptr(), mass.data_ptr(), rows, nB,
+                                 out.data_ptr(), _stream(mass))
+    check(st, "dsa_mass_to_probs")
+    return out
+
+
 def device_status(device: Optional[torch.device] = None) -> None:
     """Synchronises the current stream and raises DSAError if a kernel flagged bad input."""
     s = torch.cuda.current_stream(device).cuda_stream

@@ -13,6 +13,8 @@
  *   dsa_attn_fwd     exact softmax attention of every query in B_i over the
  *                    keys of the selected blocks, with per-block log-sums.
  *   dsa_block_mass   the exact softmax mass each selected block receives.
+ *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
+ *                    exact attention weights (the next mask of a schedule).
  *
  * Sources: "Sparse Attention for Video Generation Acceleration via Growing
  * Sparsity and Reduced Search" (GSRS, arXiv 2610.21129): abstract (Top-p
@@ -169,6 +171,31 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
 dsa_status dsa_block_mass(const float* lse, const float* blk_lse,
                           int B, int H, int N, int block, const int32_t* row_ptr,
                           float* mass, void* stream);
+
+/*
+ * Dense probability rows from the exact block masses of a CSR mask, so that
+ * dsa_select_topp can select on exact attention weights (GSRS abstract:
+ * Top-p selection supported by exact attention weights computed within the
+ * FlashAttention pass; Figure 4: later searches evaluate only the blocks of
+ * the candidate mask).
+ *
+ *   probs[r, j] = mass[s]  for every slot s of row r with col_idx[s] = j,
+ *   probs[r, j] = 0        for every other column j < nB.
+ *
+ *   row_ptr, col_idx   device, int32: the CSR mask over `rows` rows (any
+ *                      column order, no repeated column within a row).
+ *   mass      device, fp32 [nnz], aligned with col_idx (dsa_block_mass's
+ *             output; over a row the masses sum to 1).
+ *   rows, nB  rows >= 1, 1 <= nB <= DSA_MAX_BLOCKS.
+ *   probs     device out, fp32 [rows, nB].
+ * Passing probs with the same CSR as candidates to dsa_select_topp keeps
+ * the shortest prefix of each row's blocks, by exact mass, reaching p.
+ * Errors: DSA_ERR_INVALID_ARG for null or misaligned pointers and bad
+ * sizes; a column index outside [0, nB) or a decreasing row_ptr sets the
+ * device error word (dsa_device_status) and that slot or row is skipped.
+ */
+dsa_status dsa_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx, const float* mass,
+                             int rows, int nB, float* probs, void* stream);
 
 /* Largest `rows` that dsa_select_topp_static accepts. */
 #define DSA_STATIC_MAX_ROWS 32768

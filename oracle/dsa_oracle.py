@@ -213,6 +213,20 @@ def block_mass(lse, blk_lse, row_ptr, N: int, Bs: int) -> np.ndarray:
     return M
 
 
+def mass_rows(row_ptr, col, mass, nB: int) -> np.ndarray:
+    """Dense rows [rows, nB] holding each slot's exact block mass at its
+    column and 0 elsewhere.  GSRS abstract: Top-p selection on exact
+    attention weights; Figure 4: later searches evaluate only the candidate
+    mask -- so these rows, with the same CSR as candidates, are the input of
+    a mass-driven reselection (topp_select with cand)."""
+    rows = len(row_ptr) - 1
+    out = np.zeros((rows, nB), dtype=np.float64)
+    for r in range(rows):
+        for s in range(int(row_ptr[r]), int(row_ptr[r + 1])):
+            out[r, int(col[s])] = float(mass[s])
+    return out
+
+
 def dense_attention(q, k, v, scale: float):
     """Textbook softmax(scale * Q K^T) V over all N keys, fp64; also lse."""
     q = np.asarray(q, np.float64)

@@ -114,6 +114,14 @@ def test_attn_and_mass_reject(lib):
     assert lib.dsa_block_mass(FAKE, FAKE, 1, 2, 256, 100, FAKE, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
 
 
+def test_mass_to_probs_rejects(lib):
+    assert lib.dsa_mass_to_probs(None, FAKE, FAKE, 4, 4, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_mass_to_probs(FAKE, FAKE, FAKE, 0, 4, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_mass_to_probs(FAKE, FAKE, FAKE, 4, 0, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_mass_to_probs(FAKE, FAKE, FAKE, 4, 2000, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_mass_to_probs(FAKE, FAKE, FAKE + 2, 4, 4, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+
+
 def test_python_wrapper_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_lib, "_lib", None)

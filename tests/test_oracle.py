@@ -274,6 +274,53 @@ def test_block_mass_sums_to_one_and_matches_dense_weights():
     np.testing.assert_allclose(M, dense, rtol=1e-12)
 
 
+def test_mass_rows_closed_form():
+    # two rows of a 5-block mask, columns in any order
+    rp = np.array([0, 3, 5])
+    col = np.array([4, 0, 2, 1, 3])
+    mass = np.array([0.5, 0.25, 0.25, 0.75, 0.25])
+    R = O.mass_rows(rp, col, mass, 5)
+    np.testing.assert_array_equal(R, [[0.25, 0.0, 0.25, 0.0, 0.5], [0.0, 0.75, 0.0, 0.25, 0.0]])
+
+
+def test_mass_reselection_is_topp_of_dense_block_weights():
+    # Top-p on the exact masses from an all-blocks pass equals, by brute
+    # force over all subsets of the block weights of the textbook softmax
+    # matrix, the heaviest subset among the smallest ones reaching p; within
+    # a candidate mask, p = 1 keeps the mask and the result is always a
+    # subset of it.
+    N, Bs, D, scale = 384, 64, 8, 0.6
+    q, k, v = _qkv(N, D, 11, scale=1.2)
+    nB = 6
+    rp, col = _all_blocks(nB)
+    _, lse, blk = O.sparse_attention_head(q, k, v, Bs, scale, rp, col)
+    M = O.block_mass(lse, blk, rp, N, Bs)
+    P = O.mass_rows(rp, col, M, nB).astype(np.float32)
+    z = scale * q @ k.T
+    w = np.exp(z - z.max(1, keepdims=True))
+    w /= w.sum(1, keepdims=True)
+    b = O.block_bounds(N, Bs)
+    W = np.array([[w[a0:a1, c0:c1].sum(1).mean() for (c0, c1) in b] for (a0, a1) in b])
+    for p in (0.5, 0.8, 0.95):
+        srp, scol = O.topp_select(P, p, rp, col)
+        for i in range(nB):
+            best = None
+            for size in range(1, nB + 1):
+                ok = [sub for sub in itertools.combinations(range(nB), size)
+                      if W[i, list(sub)].sum() >= p]
+                if ok:
+                    best = max(ok, key=lambda sub: W[i, list(sub)].sum())
+                    break
+            np.testing.assert_array_equal(scol[srp[i]:srp[i + 1]], sorted(best))
+    cand_rp, cand_col = O.topp_select(P, 0.9, rp, col)
+    keep_rp, keep_col = O.topp_select(P, 1.0, cand_rp, cand_col)
+    np.testing.assert_array_equal(keep_rp, cand_rp)
+    np.testing.assert_array_equal(keep_col, cand_col)
+    sub_rp, sub_col = O.topp_select(P, 0.6, cand_rp, cand_col)
+    for i in range(nB):
+        assert set(sub_col[sub_rp[i]:sub_rp[i + 1]]) <= set(cand_col[cand_rp[i]:cand_rp[i + 1]])
+
+
 def test_recall_is_one_at_p1_and_pipeline_reduced_equals_full():
     N, Bs, D = 256, 64, 8
     q, k, v = _qkv(N, D, 9, scale=1.5)
