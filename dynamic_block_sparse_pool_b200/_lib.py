@@ -29,6 +29,8 @@ SIGNATURES = {
     "dsa_attn_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
     "dsa_block_mass": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "dsa_mass_to_probs": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
+    "dsa_hilbert_order": (_i, [_i, _i, _i, _i, _vp]),
+    "dsa_permute_tokens": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp]),
     "dsa_select_topp_static": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]),
     "dsa_device_status": (_i, [_vp]),
     "dsa_last_error": (ctypes.c_char_p, []),

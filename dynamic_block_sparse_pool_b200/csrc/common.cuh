@@ -14,6 +14,7 @@ enum : unsigned {
   kErrProb = 4u,         // a probability outside [0, 1] or NaN
   kErrTimeout = 8u,      // a bounded wait on an mbarrier ran out
   kErrAlign = 16u,       // dynamic shared memory not 1024-byte aligned
+  kErrPerm = 32u,        // a token permutation entry outside [0, N)
 };
 
 // Upper bound for one mbarrier wait before a kernel gives up (nanoseconds).
@@ -59,6 +60,11 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int B
 cudaError_t launch_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx,
                                  const float* mass, int rows, int nB, float* probs,
                                  unsigned* err, cudaStream_t s);
+// Index of grid cell (t, y, x) along the 3-D Hilbert curve of side 2^bits (host).
+uint64_t hilbert_key3(uint32_t t, uint32_t y, uint32_t x, int bits);
+cudaError_t launch_permute_tokens(const void* src, void* dst, int elem_bytes, int BH, int N,
+                                  int D, const int32_t* perm, bool inverse, unsigned* err,
+                                  cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

@@ -1,6 +1,9 @@
 // C ABI of libdsa (declared in include/dsa.h): argument checks, error
 // reporting and dispatch to the kernel launchers.  No call allocates device
 // memory or synchronises the host, except dsa_device_status.
+#include <algorithm>
+#include <utility>
+#include <vector>
 #include <climits>
 #include <cstdarg>
 #include <cmath>
@@ -239,6 +242,51 @@ dsa_status dsa_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx, con
   return DSA_OK;
 }
 
+dsa_status dsa_hilbert_order(int T, int H, int W, int n_prefix, int32_t* perm) {
+  g_last_error.clear();
+  if (!perm) return fail(DSA_ERR_INVALID_ARG, "null perm");
+  if (T < 1 || H < 1 || W < 1 || n_prefix < 0)
+    return fail(DSA_ERR_INVALID_ARG, "need T, H, W >= 1 and n_prefix >= 0");
+  const int side = std::max(T, std::max(H, W));
+  if (side > (1 << 20)) return fail(DSA_ERR_INVALID_ARG, "grid side above 2^20");
+  const long long cells = (long long)T * H * W;
+  if (cells + n_prefix > 0x7fffffffLL) return fail(DSA_ERR_INVALID_ARG, "too many tokens");
+  int bits = 1;
+  while ((1 << bits) < side) ++bits;
+  std::vector<std::pair<uint64_t, int32_t>> keys;
+  keys.reserve((size_t)cells);
+  for (int t = 0; t < T; ++t)
+    for (int y = 0; y < H; ++y)
+      for (int x = 0; x < W; ++x)
+        keys.emplace_back(dsa::hilbert_key3((uint32_t)t, (uint32_t)y, (uint32_t)x, bits),
+                          (int32_t)(n_prefix + ((long long)t * H + y) * W + x));
+  std::sort(keys.begin(), keys.end());
+  for (int i = 0; i < n_prefix; ++i) perm[i] = i;
+  for (size_t i = 0; i < keys.size(); ++i) perm[n_prefix + i] = keys[i].second;
+  return DSA_OK;
+}
+
+dsa_status dsa_permute_tokens(const void* src, void* dst, dsa_dtype dt, int B, int H, int N, int D,
+                              const int32_t* perm, int inverse, void* stream) {
+  g_last_error.clear();
+  if (!src || !dst || !perm) return fail(DSA_ERR_INVALID_ARG, "null src, dst or perm");
+  if (src == dst) return fail(DSA_ERR_INVALID_ARG, "src and dst must differ");
+  if (dt != DSA_F32 && dt != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (B < 1 || H < 1 || N < 1) return fail(DSA_ERR_INVALID_ARG, "need B, H, N >= 1");
+  if (D != 64 && D != 128) return fail(DSA_ERR_INVALID_ARG, "D must be 64 or 128 (got %d)", D);
+  if (inverse != 0 && inverse != 1) return fail(DSA_ERR_INVALID_ARG, "inverse must be 0 or 1");
+  if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(perm, 4))
+    return fail(DSA_ERR_INVALID_ARG, "src and dst must be 16-byte aligned, perm 4-byte aligned");
+  DeviceInfo* dev = nullptr;
+  dsa_status st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  cudaError_t e = dsa::launch_permute_tokens(src, dst, dt == DSA_BF16 ? 2 : 4, B * H, N, D, perm,
+                                             inverse != 0, dev->err_word,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "permute_tokens launch");
+  return DSA_OK;
+}
+
 dsa_status dsa_device_status(void* stream) {
   g_last_error.clear();
   DeviceInfo* dev = nullptr;
@@ -253,11 +301,12 @@ dsa_status dsa_device_status(void* stream) {
   const unsigned zero = 0;
   e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
   if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
-  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s", word,
+  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s%s", word,
               (word & dsa::kErrCsrIndex) ? " csr-index-out-of-range" : "",
               (word & dsa::kErrRowPtr) ? " bad-row-ptr" : "",
               (word & dsa::kErrProb) ? " probability-outside-[0,1]" : "",
-              (word & dsa::kErrTimeout) ? " wait-timeout" : "");
+              (word & dsa::kErrTimeout) ? " wait-timeout" : "",
+              (word & dsa::kErrPerm) ? " permutation-index-out-of-range" : "");
 }
 
 }  // extern "C"

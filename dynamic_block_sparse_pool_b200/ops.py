@@ -163,6 +163,47 @@ def mass_to_probs(row_ptr: torch.Tensor, col_idx: torch.Tensor, mass: torch.Tens
     return out
 
 
+def hilbert_order(T: int, H: int, W: int, n_prefix: int = 0) -> torch.Tensor:
+    """Host int32 [n_prefix + T*H*W]: perm[i] = original index of the token at
+    position i along the 3-D Hilbert curve (text prefix first)."""
+    perm = torch.empty(n_prefix + T * H * W, dtype=torch.int32)
+    check(lib().dsa_hilbert_order(T, H, W, n_prefix, perm.data_ptr()), "dsa_hilbert_order")
+    return perm
+
+
+def permute_tokens(x: torch.Tensor, perm: torch.Tensor, inverse: bool = False,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Gather (dst[i] = src[perm[i]]) or scatter (dst[perm[i]] = src[i]) of the
+    token rows of x [B, H, N, D]; perm: device int32 [N]."""
+    if x.dim() != 4 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor [B, H, N, D]")
+    B, H, N, D = x.shape
+    if perm.dtype != torch.int32 or not perm.is_cuda or perm.numel() != N:
+        raise ValueError("perm must be a device int32 tensor of N entries")
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib().dsa_permute_tokens(x.data_ptr(), out.data_ptr(), _dtype_code(x), B, H, N, D,
+                                  perm.data_ptr(), 1 if inverse else 0, _stream(x))
+    check(st, "dsa_permute_tokens")
+    return out
+
+
+class HilbertOrder:
+    """The Hilbert token order of one grid, kept on the device."""
+
+    def __init__(self, T: int, H: int, W: int, n_prefix: int = 0, device=None):
+        self.host = hilbert_order(T, H, W, n_prefix)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        self.perm = self.host.to(dev)
+
+    def gather(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        return permute_tokens(x, self.perm, False, out)
+
+    def scatter(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        return permute_tokens(x, self.perm, True, out)
+
+
 def device_status(device: Optional[torch.device] = None) -> None:
     """Synchronises the current stream and raises DSAError if a kernel flagged bad input."""
     s = torch.cuda.current_stream(device).cuda_stream

@@ -15,6 +15,8 @@
  *   dsa_block_mass   the exact softmax mass each selected block receives.
  *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
  *                    exact attention weights (the next mask of a schedule).
+ *   dsa_hilbert_order, dsa_permute_tokens  token reordering along a 3-D
+ *                    Hilbert curve before the pipeline, and back after it.
  *
  * Sources: "Sparse Attention for Video Generation Acceleration via Growing
  * Sparsity and Reduced Search" (GSRS, arXiv 2610.21129): abstract (Top-p
@@ -196,6 +198,43 @@ dsa_status dsa_block_mass(const float* lse, const float* blk_lse,
  */
 dsa_status dsa_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx, const float* mass,
                              int rows, int nB, float* probs, void* stream);
+
+/*
+ * Token order along a 3-D Hilbert curve (GSRS Figure 6: a block then holds
+ * the tokens of a compact spatio-temporal region instead of a flat slab;
+ * Figures 1 and 3 and the DFSAttn abstract reorder tokens along Hilbert
+ * curves).  Host function, no device work.
+ *
+ *   perm[i] = the original index of the token placed at position i.
+ *   The text prefix keeps positions 0 .. n_prefix-1; grid token (t, y, x),
+ *   original index n_prefix + (t*H + y)*W + x, is placed by its index along
+ *   the Hilbert curve of the enclosing cube of side 2^bits (Skilling's
+ *   axes-to-transpose method, t the most significant axis); cells outside
+ *   the grid are skipped.
+ *
+ *   perm   host out, int32 [n_prefix + T*H*W].
+ * Errors: DSA_ERR_INVALID_ARG for a null perm, T, H or W < 1, n_prefix < 0,
+ * a side above 2^20 or more than 2^31 - 1 tokens.
+ */
+dsa_status dsa_hilbert_order(int T, int H, int W, int n_prefix, int32_t* perm);
+
+/*
+ * Reorders whole token rows of a [B, H, N, D] tensor by a permutation of N:
+ *   inverse = 0 (gather):  dst[b, h, i, :] = src[b, h, perm[i], :]
+ *   inverse = 1 (scatter): dst[b, h, perm[i], :] = src[b, h, i, :]
+ * so gathering Q, K, V with dsa_hilbert_order's perm, running the pipeline
+ * and scattering O gives the attention of the original token order with
+ * blocks drawn along the curve.
+ *
+ *   src, dst   device, contiguous [B, H, N, D], distinct, 16-byte aligned.
+ *   perm       device, int32 [N], a permutation of 0 .. N-1.
+ * Errors: DSA_ERR_INVALID_ARG for null, aliased or misaligned pointers, an
+ * unknown dtype, D not in {64, 128} or B, H, N < 1; an entry of perm
+ * outside [0, N) sets the device error word (dsa_device_status) and that
+ * row is not copied.
+ */
+dsa_status dsa_permute_tokens(const void* src, void* dst, dsa_dtype dt, int B, int H, int N, int D,
+                              const int32_t* perm, int inverse, void* stream);
 
 /* Largest `rows` that dsa_select_topp_static accepts. */
 #define DSA_STATIC_MAX_ROWS 32768

@@ -227,6 +227,63 @@ def mass_rows(row_ptr, col, mass, nB: int) -> np.ndarray:
     return out
 
 
+def hilbert_index3(t: int, y: int, x: int, bits: int) -> int:
+    """Position of cell (t, y, x) along the 3-D Hilbert curve of the cube of
+    side 2^bits: Skilling's axes-to-transpose method ("Programming the
+    Hilbert curve", 2004) followed by interleaving the bits of the
+    transposed coordinates, most significant first, t before y before x.
+    (GSRS Figure 6 and DFSAttn abstract: tokens reordered along a Hilbert
+    curve so that a block covers a compact spatio-temporal region.)"""
+    X = [t, y, x]
+    n = 3
+    top = 1 << (bits - 1)
+    # undo the excess work: for each bit from the top, invert or exchange
+    q = top
+    while q > 1:
+        low = q - 1
+        for i in range(n):
+            if X[i] & q:
+                X[0] ^= low
+            else:
+                swap = (X[0] ^ X[i]) & low
+                X[0] ^= swap
+                X[i] ^= swap
+        q >>= 1
+    # Gray encode
+    for i in range(1, n):
+        X[i] ^= X[i - 1]
+    flip = 0
+    q = top
+    while q > 1:
+        if X[n - 1] & q:
+            flip ^= q - 1
+        q >>= 1
+    for i in range(n):
+        X[i] ^= flip
+    # interleave: bit b of X[0], X[1], X[2], for b from the top down
+    h = 0
+    for b in range(bits - 1, -1, -1):
+        for i in range(n):
+            h = (h << 1) | ((X[i] >> b) & 1)
+    return h
+
+
+def hilbert_order(T: int, H: int, W: int, n_prefix: int = 0) -> np.ndarray:
+    """perm [n_prefix + T*H*W]: perm[i] = original index of the token placed
+    at position i.  The text prefix keeps positions 0 .. n_prefix - 1; grid
+    token (t, y, x) (original index n_prefix + (t*H + y)*W + x) is placed by
+    its Hilbert index on the enclosing power-of-two cube (cells outside the
+    grid are skipped)."""
+    bits = max(1, max(T, H, W) - 1).bit_length()
+    keys = []
+    for t in range(T):
+        for y in range(H):
+            for x in range(W):
+                keys.append((hilbert_index3(t, y, x, bits), n_prefix + (t * H + y) * W + x))
+    keys.sort()
+    return np.array(list(range(n_prefix)) + [idx for _, idx in keys], dtype=np.int64)
+
+
 def dense_attention(q, k, v, scale: float):
     """Textbook softmax(scale * Q K^T) V over all N keys, fp64; also lse."""
     q = np.asarray(q, np.float64)

@@ -338,3 +338,46 @@ def test_executed_flops_counts_ragged_blocks():
     rp = np.array([0, 2, 3])
     col = np.array([0, 1, 1])          # N = 100, Bs = 64: blocks of 64 and 36
     assert O.executed_flops(rp, col, 100, 64, 8) == 4 * 8 * (64 * 64 + 64 * 36 + 36 * 36)
+
+
+# --------------------------------------------------------- Hilbert order ----
+
+def _cells(perm, H, W, n_prefix=0):
+    g = np.asarray(perm[n_prefix:]) - n_prefix
+    return np.stack([g // (H * W), (g // W) % H, g % W], axis=1)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_hilbert_cube_is_a_unit_step_path_with_adjacent_ends(bits):
+    n = 1 << bits
+    perm = O.hilbert_order(n, n, n)
+    assert sorted(perm.tolist()) == list(range(n ** 3))
+    c = _cells(perm, n, n)
+    steps = np.abs(np.diff(c, axis=0)).sum(1)
+    assert np.all(steps == 1)                       # continuity of the curve
+    assert tuple(c[0]) == (0, 0, 0)
+    end = c[-1]                                     # the 3-D curve ends at an adjacent corner
+    assert sorted(end.tolist()) == [0, 0, n - 1]
+
+
+def test_hilbert_subgrid_is_the_cube_order_filtered_and_prefix_is_kept():
+    T, H, W, P = 3, 5, 6, 4
+    perm = O.hilbert_order(T, H, W, P)
+    assert perm[:P].tolist() == list(range(P))
+    assert sorted(perm.tolist()) == list(range(P + T * H * W))
+    cube = _cells(O.hilbert_order(8, 8, 8), 8, 8)
+    inside = [tuple(c) for c in cube if c[0] < T and c[1] < H and c[2] < W]
+    assert [tuple(c) for c in _cells(perm, H, W, P)] == inside
+
+
+def test_hilbert_blocks_are_more_compact_than_row_major():
+    T, H, W, Bs = 6, 12, 20, 64
+    perm = O.hilbert_order(T, H, W)
+    def extent(order):
+        c = _cells(order, H, W)
+        ext = []
+        for a in range(0, len(order), Bs):
+            blk = c[a:a + Bs]
+            ext.append(np.prod(blk.max(0) - blk.min(0) + 1))
+        return float(np.mean(ext))
+    assert extent(perm) < 0.5 * extent(np.arange(T * H * W))
