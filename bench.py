@@ -312,7 +312,7 @@ def sweep(args):
         reps = max(3, int(seconds * 1e3 / max(est_ms, 1e-2)))
         return timed(lambda: [fn() for _ in range(reps)], 1) / reps
 
-    def point(w, q, k, v, p, cand=None, dense=None, label=None, extra=None):
+    def point(w, q, k, v, p, cand=None, dense=None, label=None, extra=None, hier_sub=None):
         B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
         nB, rows = w.n_blocks, w.BH * w.n_blocks
         scale = 1.0 / math.sqrt(D)
@@ -326,7 +326,13 @@ def sweep(args):
         cap = rows * nB if cand is None else int(cand[0][-1])
         bl = torch.empty(max(cap, 1), blk, device=dev)
         ms_ = torch.empty(max(cap, 1), device=dev)
-        search = lambda: (ops.pool_score(q, k, blk, scale, cand=cand, out=P, workspace=wp),
+        if hier_sub is not None:
+            wh = torch.empty(ops.workspace_size(2 if hier_sub <= 2 else 3, B, H, N, D, blk),
+                             device=dev, dtype=torch.uint8)
+            score = lambda: ops.pool_score_hier(q, k, blk, hier_sub, scale, out=P, workspace=wh)
+        else:
+            score = lambda: ops.pool_score(q, k, blk, scale, cand=cand, out=P, workspace=wp)
+        search = lambda: (score(),
                           ops.select_topp(P, p, cand=cand, row_ptr=rp, col_idx=ci, workspace=wsel))
         attend = lambda: ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=bl)
         mass = lambda: ops.block_mass(lse, bl, rp, blk, mass=ms_)
@@ -385,6 +391,8 @@ def sweep(args):
     masks = {}
     for p in w.p:
         masks[p] = point(w, q, k, v, p, dense=dms)[:2]
+    # the same point with the two-level (sub-block) estimate
+    point(w, q, k, v, 0.9, dense=dms, label=w.name + " two-level estimate (sub 2)", hier_sub=2)
     # the same point on Hilbert-ordered tokens (dense attention is order-free),
     # plus the cost of gathering Q, K, V and scattering O
     order = ops.HilbertOrder(w.T, w.Hg, w.W, w.n_prefix, device=dev)

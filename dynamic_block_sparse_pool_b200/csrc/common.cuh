@@ -65,6 +65,8 @@ uint64_t hilbert_key3(uint32_t t, uint32_t y, uint32_t x, int bits);
 cudaError_t launch_permute_tokens(const void* src, void* dst, int elem_bytes, int BH, int N,
                                   int D, const int32_t* perm, bool inverse, unsigned* err,
                                   cudaStream_t s);
+cudaError_t launch_aggregate_probs(const float* pf, int BH, int N, int block, int sub, int nB,
+                                   int nBf, float* probs, cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

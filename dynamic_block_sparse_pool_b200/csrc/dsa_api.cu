@@ -100,6 +100,11 @@ bool cand_ok(const int32_t* rp, const int32_t* col) { return (rp == nullptr) == 
 
 size_t pool_ws_bytes(long long BH, long long nB, int D) { return (size_t)(2 * BH * nB * D) * sizeof(float); }
 size_t select_ws_bytes(long long rows) { return (size_t)(rows * 33) * sizeof(uint32_t); }
+// fine means (2 * BH * nBf * D floats) and the fine row softmax (BH * nBf^2 floats)
+size_t hier_ws_bytes(long long BH, long long nBf, int D) {
+  return (size_t)(2 * BH * nBf * D + BH * nBf * nBf) * sizeof(float);
+}
+constexpr int kMaxFineBlocks = 2048;  // the score kernel's tile mask covers 32 tiles of 64
 
 }  // namespace
 
@@ -115,6 +120,11 @@ size_t dsa_workspace_size(int op, int B, int H, int N, int D, int block) {
   const long long BH = (long long)B * H;
   if (op == DSA_OP_POOL_SCORE) return pool_ws_bytes(BH, nB, D);
   if (op == DSA_OP_SELECT_TOPP) return select_ws_bytes(BH * nB);
+  if (op == DSA_OP_POOL_SCORE_HIER2 || op == DSA_OP_POOL_SCORE_HIER4) {
+    const int sub = op == DSA_OP_POOL_SCORE_HIER2 ? 2 : 4;
+    const long long bf = block / sub;
+    return hier_ws_bytes(BH, (N + bf - 1) / bf, D);
+  }
   return 0;
 }
 
@@ -146,6 +156,44 @@ dsa_status dsa_pool_score(const void* q, const void* k, dsa_dtype dt, int B, int
   e = dsa::launch_block_scores(qbar, kbar, (int)BH, nB, D, scale, cand_row_ptr, cand_col, probs,
                                dev->err_word, s);
   if (e != cudaSuccess) return cuda_fail(e, "block_scores launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_pool_score_hier(const void* q, const void* k, dsa_dtype dt, int B, int H, int N,
+                               int D, int block, int sub, float scale, float* probs,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !probs || !workspace) return fail(DSA_ERR_INVALID_ARG, "null q, k, probs or workspace");
+  if (dt != DSA_F32 && dt != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  dsa_status st = check_shape(B, H, N, D, block);
+  if (st != DSA_OK) return st;
+  if (sub != 1 && sub != 2 && sub != 4) return fail(DSA_ERR_INVALID_ARG, "sub must be 1, 2 or 4 (got %d)", sub);
+  const int nB = (N + block - 1) / block;
+  const int bf = block / sub;
+  const int nBf = (N + bf - 1) / bf;
+  const long long BH = (long long)B * H;
+  if ((st = check_blocks_limit(BH * nB, nB)) != DSA_OK) return st;
+  if (nBf > kMaxFineBlocks)
+    return fail(DSA_ERR_INVALID_ARG, "%d sub-blocks per row; at most %d supported", nBf, kMaxFineBlocks);
+  if (BH * nBf * nBf >= INT_MAX) return fail(DSA_ERR_INVALID_ARG, "fine score matrix too large");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(probs, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q, k and workspace must be 16-byte aligned, probs 4-byte aligned");
+  if (ws_bytes < hier_ws_bytes(BH, nBf, D))
+    return fail(DSA_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes, hier_ws_bytes(BH, nBf, D));
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* qbar = static_cast<float*>(workspace);
+  float* kbar = qbar + BH * nBf * D;
+  float* pf = kbar + BH * nBf * D;
+  cudaError_t e = dsa::launch_pool_means(q, k, dt == DSA_BF16, (int)BH, N, D, bf, qbar, kbar, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pool_means launch");
+  e = dsa::launch_block_scores(qbar, kbar, (int)BH, nBf, D, scale, nullptr, nullptr, pf,
+                               dev->err_word, s);
+  if (e != cudaSuccess) return cuda_fail(e, "block_scores launch");
+  e = dsa::launch_aggregate_probs(pf, (int)BH, N, block, sub, nB, nBf, probs, s);
+  if (e != cudaSuccess) return cuda_fail(e, "aggregate_probs launch");
   return DSA_OK;
 }
 

@@ -9,6 +9,10 @@
 // Kernel 1 (pool_means): one CTA per (block, head, Q-or-K); 16-byte loads,
 //   fp32 accumulation, mean over the block's actual rows.  HBM-bound: reads
 //   Q and K once.
+// Two-level estimate (DFSAttn abstract: hierarchical block scoring): the
+//   two kernels above at sub-block granularity, then aggregate_probs folds
+//   the fine row softmax back into block rows (token-weighted over query
+//   sub-blocks, summed over key sub-blocks).
 // Kernel 2 (block_scores): one CTA per (64 query-block rows, head): a
 //   register-tiled fp32 product of the 64 pooled queries with double-buffered
 //   tiles of 64 pooled keys (cp.async), scaled scores written to P with a
@@ -279,6 +283,36 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
   }
 }
 
+// Block rows of the two-level estimate from the fine (sub-block) row softmax
+// pf [BH, nBf, nBf]: P[i, j] = sum over the query sub-blocks a of block i of
+// (|a| / |B_i|) * (sum of pf[a, b] over the key sub-blocks b of block j).
+// One warp per block row, lanes over block columns; each fine value is read
+// once.
+__global__ void __launch_bounds__(256)
+aggregate_probs_kernel(const float* __restrict__ pf, int N, int block, int sub, int nB, int nBf,
+                       float* __restrict__ probs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + warp;
+  const int bh = blockIdx.y;
+  if (i >= nB) return;
+  const int bf = block / sub;
+  const int i0 = i * block;
+  const float inv_len = 1.0f / (float)min(block, N - i0);
+  const float* fhead = pf + (size_t)bh * nBf * nBf;
+  float* prow = probs + ((size_t)bh * nB + i) * nB;
+  for (int j = lane; j < nB; j += 32) {
+    float acc = 0.f;
+    for (int a = i * sub; a < min((i + 1) * sub, nBf); ++a) {
+      const float w = (float)min(bf, N - a * bf) * inv_len;
+      const float* frow = fhead + (size_t)a * nBf;
+      float part = 0.f;
+      for (int b = j * sub; b < min((j + 1) * sub, nBf); ++b) part += frow[b];
+      acc = fmaf(w, part, acc);
+    }
+    prow[j] = acc;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_pool_means(const void* q, const void* k, bool bf16, int BH, int N,
@@ -320,6 +354,16 @@ cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, in
   if (D == 64)
     return launch_scores_d<64>(qbar, kbar, BH, nB, scale, cand_row_ptr, cand_col, probs, err, s);
   return launch_scores_d<128>(qbar, kbar, BH, nB, scale, cand_row_ptr, cand_col, probs, err, s);
+}
+
+}  // namespace dsa
+
+namespace dsa {
+
+cudaError_t launch_aggregate_probs(const float* pf, int BH, int N, int block, int sub, int nB,
+                                   int nBf, float* probs, cudaStream_t s) {
+  aggregate_probs_kernel<<<dim3(ceil_div(nB, 8), BH), 256, 0, s>>>(pf, N, block, sub, nB, nBf, probs);
+  return cudaGetLastError();
 }
 
 }  // namespace dsa

@@ -85,6 +85,28 @@ def pool_score(q: torch.Tensor, k: torch.Tensor, block: int, scale: Optional[flo
     return out
 
 
+def pool_score_hier(q: torch.Tensor, k: torch.Tensor, block: int, sub: int,
+                    scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """P [B*H, nB, nB] fp32: the two-level estimate (pooled scores over
+    sub-blocks of block/sub rows, folded back into block rows); sub = 1 is
+    pool_score's P."""
+    B, H, N, D = _check_qkv(q, k)
+    nB = n_blocks(N, block)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(B * H, nB, nB, device=q.device, dtype=torch.float32)
+    op = _lib.DSA_OP_POOL_SCORE_HIER4 if sub == 4 else _lib.DSA_OP_POOL_SCORE_HIER2
+    ws_bytes = workspace_size(op, B, H, N, D, block)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
+    st = lib().dsa_pool_score_hier(q.data_ptr(), k.data_ptr(), _dtype_code(q), B, H, N, D, block,
+                                   sub, scale, out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _stream(q))
+    check(st, "dsa_pool_score_hier")
+    return out
+
+
 def select_topp(probs: torch.Tensor, p: float, cand: Optional[Csr] = None,
                 row_ptr: Optional[torch.Tensor] = None, col_idx: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None) -> Csr:

@@ -73,7 +73,8 @@ typedef enum dsa_status {
 typedef enum dsa_dtype { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
 
 /* Operation ids for dsa_workspace_size. */
-enum { DSA_OP_POOL_SCORE = 0, DSA_OP_SELECT_TOPP = 1 };
+enum { DSA_OP_POOL_SCORE = 0, DSA_OP_SELECT_TOPP = 1, DSA_OP_POOL_SCORE_HIER2 = 2,
+       DSA_OP_POOL_SCORE_HIER4 = 3 };
 
 /* Largest number of blocks per row that dsa_pool_score / dsa_select_topp
  * accept (one warp sorts a row of up to 1024 blocks in registers). */
@@ -84,6 +85,9 @@ enum { DSA_OP_POOL_SCORE = 0, DSA_OP_SELECT_TOPP = 1 };
  * block as in the calls below).  Returns 0 for invalid sizes.
  *   DSA_OP_POOL_SCORE : 2 * B*H*nB*D floats (pooled means).
  *   DSA_OP_SELECT_TOPP: B*H*nB * 33 words (selection bitmaps and counts).
+ *   DSA_OP_POOL_SCORE_HIER2 / _HIER4: dsa_pool_score_hier with sub = 2 / 4:
+ *     2 * B*H*nBf*D floats (sub-block means) + B*H*nBf^2 floats (their row
+ *     softmax), nBf = ceil(N / (block / sub)).
  */
 size_t dsa_workspace_size(int op, int B, int H, int N, int D, int block);
 
@@ -109,6 +113,27 @@ dsa_status dsa_pool_score(const void* q, const void* k, dsa_dtype dt,
                           const int32_t* cand_row_ptr, const int32_t* cand_col,
                           float* probs, void* workspace, size_t ws_bytes,
                           void* stream);
+
+/*
+ * Two-level block estimate (DFSAttn abstract: hierarchical block scoring for
+ * block importance; the pages give no construction, so this is the plain
+ * two-level pooling): the block means and row softmax of dsa_pool_score,
+ * taken over sub-blocks of block/sub rows, then folded back into block rows.
+ *
+ *   Pf[a, b] = softmax_b(scale * qbar_a . kbar_b) over the sub-blocks,
+ *   probs[i, j] = sum over the query sub-blocks a of block i of
+ *                 (|a| / |B_i|) * sum over the key sub-blocks b of block j of Pf[a, b].
+ *
+ * sub = 1 gives dsa_pool_score's P.  Full search only (no candidate set).
+ *   sub       1, 2 or 4 (block / sub rows per sub-block).
+ *   workspace >= dsa_workspace_size(DSA_OP_POOL_SCORE_HIER2 or _HIER4, ...)
+ *             bytes (sub = 1 needs the _HIER2 size or more), 16-byte aligned.
+ *   probs     device out, fp32 [B*H, nB, nB]; rows sum to 1.
+ * Limits: nB <= DSA_MAX_BLOCKS and at most 2048 sub-blocks per head.
+ */
+dsa_status dsa_pool_score_hier(const void* q, const void* k, dsa_dtype dt, int B, int H, int N,
+                               int D, int block, int sub, float scale, float* probs,
+                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Per-row Top-p block selection (GSRS abstract: Top-p selection for

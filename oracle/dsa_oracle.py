@@ -92,6 +92,35 @@ def block_probs(qbar: np.ndarray, kbar: np.ndarray, scale: float,
     return P
 
 
+def hier_block_probs(q: np.ndarray, k: np.ndarray, Bs: int, sub: int, scale: float) -> np.ndarray:
+    """Two-level block estimate (DFSAttn abstract: hierarchical block scoring
+    for block importance; the pages give no construction, this is the plain
+    two-level pooling).  Tokens are pooled over sub-blocks of Bs/sub rows;
+    each query sub-block a takes the row softmax of scale * qbar_a . kbar_b
+    over all key sub-blocks b; block row i is the token-weighted mean over
+    its query sub-blocks of the mass falling in each key block j:
+
+        P_ij = sum_{a in i} (|a| / |B_i|) sum_{b in j} softmax_b(...)_ab.
+
+    sub = 1 is block_probs."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    N = q.shape[0]
+    bf = Bs // sub
+    Pf = block_probs(pool_blocks(q, bf), pool_blocks(k, bf), scale)
+    fine = block_bounds(N, bf)
+    coarse = block_bounds(N, Bs)
+    P = np.zeros((len(coarse), len(coarse)))
+    for i, (i0, i1) in enumerate(coarse):
+        for a, (a0, a1) in enumerate(fine):
+            if i0 <= a0 < i1:
+                w = (a1 - a0) / (i1 - i0)
+                for j, (j0, j1) in enumerate(coarse):
+                    cols = [b for b, (b0, _) in enumerate(fine) if j0 <= b0 < j1]
+                    P[i, j] += w * Pf[a, cols].sum()
+    return P
+
+
 # ---------------------------------------------------------------------------
 # 3. Top-p selection (exact)
 # ---------------------------------------------------------------------------

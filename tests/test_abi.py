@@ -122,6 +122,17 @@ def test_mass_to_probs_rejects(lib):
     assert lib.dsa_mass_to_probs(FAKE, FAKE, FAKE + 2, 4, 4, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
 
 
+def test_pool_score_hier_rejects(lib):
+    ok = (FAKE, FAKE, 1, 1, 2, 256, 64, 128, 2, 0.125, FAKE, FAKE, 1 << 30, None)
+    assert lib.dsa_pool_score_hier(None, *ok[1:]) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_pool_score_hier(*ok[:8], 3, *ok[9:]) == _lib.DSA_ERR_INVALID_ARG       # sub
+    assert lib.dsa_pool_score_hier(*ok[:12], 16, None) == _lib.DSA_ERR_INVALID_ARG        # workspace
+    big = ok[:5] + (1 << 20,) + ok[6:8] + (4,) + ok[9:]                                  # > 2048 sub-blocks
+    assert lib.dsa_pool_score_hier(*big) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_workspace_size(_lib.DSA_OP_POOL_SCORE_HIER2, 1, 2, 256, 64, 128) == \
+        4 * (2 * 2 * 4 * 64 + 2 * 4 * 4)
+
+
 def test_python_wrapper_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_lib, "_lib", None)

@@ -381,3 +381,34 @@ def test_hilbert_blocks_are_more_compact_than_row_major():
             ext.append(np.prod(blk.max(0) - blk.min(0) + 1))
         return float(np.mean(ext))
     assert extent(perm) < 0.5 * extent(np.arange(T * H * W))
+
+
+# ----------------------------------------------------- hierarchical scores ----
+
+def test_hier_probs_sub1_is_block_probs_and_rows_sum_to_one():
+    N, Bs, D = 300, 64, 8
+    q, k, _ = _qkv(N, D, 21, scale=1.3)
+    P1 = O.hier_block_probs(q, k, Bs, 1, 0.4)
+    ref = O.block_probs(O.pool_blocks(q, Bs), O.pool_blocks(k, Bs), 0.4)
+    np.testing.assert_allclose(P1, ref, rtol=1e-13, atol=1e-15)
+    for sub in (2, 4):
+        P = O.hier_block_probs(q, k, Bs, sub, 0.4)
+        np.testing.assert_allclose(P.sum(1), 1.0, rtol=1e-12)
+        assert P.shape == ref.shape and np.all(P >= 0)
+
+
+def test_hier_probs_block_constant_closed_form():
+    # tokens constant within each block: every key sub-block of block j scores
+    # s_ij, so P_ij = n_j e^{s_ij} / sum_j' n_j' e^{s_ij'} with n_j the number
+    # of key sub-blocks in block j (the ragged last block has fewer)
+    Bs, sub, D = 64, 4, 6
+    N = 3 * Bs + 20                       # last block: 20 tokens -> 2 sub-blocks of 16
+    rng = np.random.default_rng(4)
+    qv, kv = rng.normal(size=(4, D)), rng.normal(size=(4, D))
+    blk = np.minimum(np.arange(N) // Bs, 3)
+    q, k = qv[blk], kv[blk]
+    P = O.hier_block_probs(q, k, Bs, sub, 0.7)
+    n = np.array([4, 4, 4, 2])
+    s = 0.7 * qv @ kv.T
+    e = n[None, :] * np.exp(s)
+    np.testing.assert_allclose(P, e / e.sum(1, keepdims=True), rtol=1e-12)
