@@ -425,6 +425,33 @@ def sweep(args):
     del q, k, v
     torch.cuda.empty_cache()
     gsrs_run(timed)
+    backward_point(timed)
+
+
+def backward_point(timed):
+    """Backward of the attention (exact fp32 on CUDA cores) on the Wan2.1-like
+    grid with 8 heads at p = 0.9.  Algorithmic FLOPs: the five contractions
+    (Q K^T, dO V^T, dS K, dS^T Q, P^T dO) = 2.5 x the forward's executed
+    FLOPs; this kernel also recomputes Q K^T and dO V^T in its dK/dV pass."""
+    import dataclasses
+    dev = torch.device("cuda", 0)
+    w = dataclasses.replace(synth.WAN21, heads=8)
+    B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+    q, k, v = synth.make_qkv(w, 0, device="cuda")
+    scale = 1.0 / math.sqrt(D)
+    sa = ops.sparse_attention(q, k, v, 0.9, block=blk, scale=scale)
+    dO = torch.randn(q.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(1)).to(q.dtype)
+    ws = torch.empty(ops.workspace_size(4, B, H, N, D, blk), device=dev, dtype=torch.uint8)
+    f = lambda: ops.attn_bwd(q, k, v, sa.out, dO, sa.lse, sa.row_ptr, sa.col_idx, blk, scale,
+                             workspace=ws)
+    f()
+    ops.device_status(dev)
+    t = timed(f, 2)
+    fwd, nnz = executed_flops(sa.row_ptr, sa.col_idx, N, blk, D, w.n_blocks)
+    line = {"sweep": "backward (exact fp32 on CUDA cores), wan2.1-like 8 heads", "p": 0.9,
+            "nnz_blocks": nnz, "bwd_ms": t, "algorithmic_tflop": 2.5 * fwd / 1e12,
+            "bwd_tflops": 2.5 * fwd / (t * 1e-3) / 1e12, "bound": "fp32 CUDA cores"}
+    print(json.dumps(line), flush=True)
 
 
 def gsrs_run(timed):

@@ -9,10 +9,10 @@ on the first call, and a call fails loudly if it has not been built.
 """
 from . import ops, synth  # noqa: F401
 from ._lib import DSAError  # noqa: F401
-from .ops import (HilbertOrder, attn_fwd, block_mass, device_status,  # noqa: F401
+from .ops import (HilbertOrder, attn_bwd, attn_fwd, block_mass, device_status,  # noqa: F401
                   hilbert_order, mass_to_probs, permute_tokens, pool_score, pool_score_hier,
                   select_topp, sparse_attention)
 
 __all__ = ["ops", "synth", "DSAError", "pool_score", "select_topp", "attn_fwd",
            "block_mass", "mass_to_probs", "sparse_attention", "device_status",
-           "hilbert_order", "permute_tokens", "HilbertOrder", "pool_score_hier"]
+           "hilbert_order", "permute_tokens", "HilbertOrder", "pool_score_hier", "attn_bwd"]

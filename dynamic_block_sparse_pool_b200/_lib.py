@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_DEVICE = range(5)
 DSA_F32, DSA_BF16 = 0, 1
 DSA_OP_POOL_SCORE, DSA_OP_SELECT_TOPP = 0, 1
-DSA_OP_POOL_SCORE_HIER2, DSA_OP_POOL_SCORE_HIER4 = 2, 3
+DSA_OP_POOL_SCORE_HIER2, DSA_OP_POOL_SCORE_HIER4, DSA_OP_ATTN_BWD = 2, 3, 4
 DSA_MAX_BLOCKS = 1024
 DSA_STATIC_MAX_ROWS = 32768
 
@@ -29,6 +29,8 @@ SIGNATURES = {
     "dsa_select_topp": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_attn_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
     "dsa_block_mass": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "dsa_attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
+                          _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_mass_to_probs": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
     "dsa_pool_score_hier": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "dsa_hilbert_order": (_i, [_i, _i, _i, _i, _vp]),

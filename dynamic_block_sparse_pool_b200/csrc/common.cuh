@@ -67,6 +67,14 @@ cudaError_t launch_permute_tokens(const void* src, void* dst, int elem_bytes, in
                                   cudaStream_t s);
 cudaError_t launch_aggregate_probs(const float* pf, int BH, int N, int block, int sub, int nB,
                                    int nBf, float* probs, cudaStream_t s);
+// Exclusive scan of `rows` counts into row_ptr[0 .. rows] (one CTA).
+cudaError_t launch_csr_scan(const int32_t* counts, int rows, int32_t* row_ptr, cudaStream_t s);
+cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, const float* lse, bool bf16, int BH, int N, int D,
+                            int block, float scale, const int32_t* row_ptr,
+                            const int32_t* col_idx, void* dq, void* dk, void* dv,
+                            uint32_t* bitmap, int32_t* counts, int32_t* t_row_ptr,
+                            int32_t* t_col, float* delta, unsigned* err, cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

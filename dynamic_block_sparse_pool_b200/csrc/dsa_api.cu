@@ -104,7 +104,13 @@ size_t select_ws_bytes(long long rows) { return (size_t)(rows * 33) * sizeof(uin
 size_t hier_ws_bytes(long long BH, long long nBf, int D) {
   return (size_t)(2 * BH * nBf * D + BH * nBf * nBf) * sizeof(float);
 }
-constexpr int kMaxFineBlocks = 2048;  // the score kernel's tile mask covers 32 tiles of 64
+constexpr int kMaxFineBlocks = 2048;
+// mask bitmap (32 words per row), counts, transposed row_ptr and column
+// capacity (rows * nB), delta (B*H*N floats)
+size_t bwd_ws_bytes(long long BH, long long nB, long long N) {
+  const long long rows = BH * nB;
+  return (size_t)(rows * 32 + rows + (rows + 1) + rows * nB + BH * N) * 4;
+}  // the score kernel's tile mask covers 32 tiles of 64
 
 }  // namespace
 
@@ -120,6 +126,7 @@ size_t dsa_workspace_size(int op, int B, int H, int N, int D, int block) {
   const long long BH = (long long)B * H;
   if (op == DSA_OP_POOL_SCORE) return pool_ws_bytes(BH, nB, D);
   if (op == DSA_OP_SELECT_TOPP) return select_ws_bytes(BH * nB);
+  if (op == DSA_OP_ATTN_BWD) return bwd_ws_bytes(BH, nB, N);
   if (op == DSA_OP_POOL_SCORE_HIER2 || op == DSA_OP_POOL_SCORE_HIER4) {
     const int sub = op == DSA_OP_POOL_SCORE_HIER2 ? 2 : 4;
     const long long bf = block / sub;
@@ -252,6 +259,42 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
                               out, lse, blk_lse, dev->err_word, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, dsa_dtype dt, int B, int H, int N,
+                        int D, int block, float scale, const int32_t* row_ptr,
+                        const int32_t* col_idx, void* dq, void* dk, void* dv, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !out || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv || !workspace)
+    return fail(DSA_ERR_INVALID_ARG, "null pointer argument");
+  if (dt != DSA_F32 && dt != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  dsa_status st = check_shape(B, H, N, D, block);
+  if (st != DSA_OK) return st;
+  const int nB = (N + block - 1) / block;
+  const long long BH = (long long)B * H;
+  if ((st = check_blocks_limit(BH * nB, nB)) != DSA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4) || !aligned(dout, 4) ||
+      !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4) || !aligned(lse, 4) ||
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(workspace, 16))
+    return fail(DSA_ERR_INVALID_ARG, "misaligned pointer");
+  if (ws_bytes < bwd_ws_bytes(BH, nB, N))
+    return fail(DSA_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes, bwd_ws_bytes(BH, nB, N));
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  const long long rows = BH * nB;
+  uint32_t* bitmap = static_cast<uint32_t*>(workspace);
+  int32_t* counts = reinterpret_cast<int32_t*>(bitmap + rows * 32);
+  int32_t* t_row_ptr = counts + rows;
+  int32_t* t_col = t_row_ptr + rows + 1;
+  float* delta = reinterpret_cast<float*>(t_col + rows * nB);
+  cudaError_t e = dsa::launch_attn_bwd(q, k, v, out, dout, lse, dt == DSA_BF16, (int)BH, N, D, block,
+                                       scale, row_ptr, col_idx, dq, dk, dv, bitmap, counts, t_row_ptr,
+                                       t_col, delta, dev->err_word, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_bwd launch");
   return DSA_OK;
 }
 

@@ -424,6 +424,11 @@ compact_kernel(const uint32_t* __restrict__ bitmaps, int rows,
 
 }  // namespace
 
+cudaError_t launch_csr_scan(const int32_t* counts, int rows, int32_t* row_ptr, cudaStream_t s) {
+  csr_scan_kernel<<<1, 1024, 0, s>>>(counts, rows, row_ptr);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const float* probs, int rows, int nB, float p,
                           const int32_t* cand_row_ptr, const int32_t* cand_col,
                           int32_t* row_ptr, int32_t* col_idx, uint32_t* bitmaps,

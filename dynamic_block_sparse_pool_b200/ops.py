@@ -158,6 +158,30 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.T
     return out, lse, blk_lse
 
 
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+             dout: torch.Tensor, lse: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+             block: int, scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None):
+    """(dQ, dK, dV) [B, H, N, D] of attn_fwd's O for a fixed mask, given dO."""
+    B, H, N, D = _check_qkv(q, k, v)
+    for t in (out, dout):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("out and dout must match q")
+    nB = n_blocks(N, block)
+    _check_csr((row_ptr, col_idx), B * H * nB)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws_bytes = workspace_size(_lib.DSA_OP_ATTN_BWD, B, H, N, D, block)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = lib().dsa_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            dout.data_ptr(), lse.data_ptr(), _dtype_code(q), B, H, N, D, block,
+                            scale, row_ptr.data_ptr(), col_idx.data_ptr(), dq.data_ptr(),
+                            dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream(q))
+    check(st, "dsa_attn_bwd")
+    return dq, dk, dv
+
+
 def block_mass(lse: torch.Tensor, blk_lse: torch.Tensor, row_ptr: torch.Tensor, block: int,
                mass: Optional[torch.Tensor] = None) -> torch.Tensor:
     """mass [nnz] (capacity blk_lse.shape[0]): exact softmax mass of each selected block."""

@@ -13,6 +13,7 @@
  *   dsa_attn_fwd     exact softmax attention of every query in B_i over the
  *                    keys of the selected blocks, with per-block log-sums.
  *   dsa_block_mass   the exact softmax mass each selected block receives.
+ *   dsa_attn_bwd     gradients of the attention for a fixed mask.
  *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
  *                    exact attention weights (the next mask of a schedule).
  *   dsa_hilbert_order, dsa_permute_tokens  token reordering along a 3-D
@@ -74,7 +75,7 @@ typedef enum dsa_dtype { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
 
 /* Operation ids for dsa_workspace_size. */
 enum { DSA_OP_POOL_SCORE = 0, DSA_OP_SELECT_TOPP = 1, DSA_OP_POOL_SCORE_HIER2 = 2,
-       DSA_OP_POOL_SCORE_HIER4 = 3 };
+       DSA_OP_POOL_SCORE_HIER4 = 3, DSA_OP_ATTN_BWD = 4 };
 
 /* Largest number of blocks per row that dsa_pool_score / dsa_select_topp
  * accept (one warp sorts a row of up to 1024 blocks in registers). */
@@ -88,6 +89,9 @@ enum { DSA_OP_POOL_SCORE = 0, DSA_OP_SELECT_TOPP = 1, DSA_OP_POOL_SCORE_HIER2 = 
  *   DSA_OP_POOL_SCORE_HIER2 / _HIER4: dsa_pool_score_hier with sub = 2 / 4:
  *     2 * B*H*nBf*D floats (sub-block means) + B*H*nBf^2 floats (their row
  *     softmax), nBf = ceil(N / (block / sub)).
+ *   DSA_OP_ATTN_BWD: 4-byte words: B*H*nB*32 (mask bitmap) + B*H*nB (counts)
+ *     + B*H*nB + 1 (transposed row_ptr) + B*H*nB*nB (transposed columns)
+ *     + B*H*N (rowsum(dO * O)).
  */
 size_t dsa_workspace_size(int op, int B, int H, int N, int D, int block);
 
@@ -185,6 +189,32 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
                         int B, int H, int N, int D, int block, float scale,
                         const int32_t* row_ptr, const int32_t* col_idx,
                         void* out, float* lse, float* blk_lse, void* stream);
+
+/*
+ * Gradients of dsa_attn_fwd's O for a fixed mask (DSV abstract: DiTs are
+ * trained with the same dynamic sparsity).  With P the softmax of each
+ * query over the keys of its row's selected blocks (from the forward's
+ * lse), dP = dO V^T and delta = rowsum(dO * O):
+ *
+ *   dS = P * (dP - delta),  dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
+ *
+ *   q, k, v, out, dout  device, [B, H, N, D] in dt (out: dsa_attn_fwd's O).
+ *   lse        device, fp32 [B, H, N]: dsa_attn_fwd's lse.
+ *   row_ptr, col_idx   the forward's CSR mask (no repeated column in a row).
+ *   dq, dk, dv device out, [B, H, N, D] in dt; key blocks that no row
+ *              selected get dK = dV = 0, queries of empty rows dQ = 0.
+ *   workspace  >= dsa_workspace_size(DSA_OP_ATTN_BWD, ...) bytes, 16-byte
+ *              aligned.
+ * Exact fp32 arithmetic on CUDA cores for both dtypes.  Every key block's
+ * contributions are summed in ascending query-block order, so the result is
+ * the same from run to run.  Errors as for dsa_attn_fwd; a malformed mask
+ * sets the device error word.
+ */
+dsa_status dsa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, dsa_dtype dt, int B, int H, int N,
+                        int D, int block, float scale, const int32_t* row_ptr,
+                        const int32_t* col_idx, void* dq, void* dk, void* dv, void* workspace,
+                        size_t ws_bytes, void* stream);
 
 /*
  * Exact softmax mass of each selected block (GSRS abstract: exact attention

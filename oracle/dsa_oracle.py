@@ -230,6 +230,52 @@ def sparse_attention_head(q, k, v, Bs: int, scale: float, row_ptr, col,
     return O, lse, blk
 
 
+def sparse_attention_backward_head(q, k, v, dO, Bs: int, scale: float, row_ptr, col, out=None):
+    """Gradients (dQ, dK, dV) [N, D] of the block-sparse attention output O
+    (as sparse_attention_head computes it, for a fixed mask) against the
+    upstream gradient dO, in fp64.  DSV abstract: attention is trained with
+    the same sparsity; this is the chain rule through each query's softmax
+    over the keys of its selected blocks:
+
+        P = softmax(scale * q K_sel^T),  dP = dO_q V_sel^T,
+        dS = P * (dP - sum(P * dP)),
+        dQ_q = scale * dS K_sel,  dK_sel += scale * dS^T q,  dV_sel += P^T dO_q.
+
+    Queries of an empty row get dQ = 0 and add nothing to dK, dV.
+
+    out: if given, the stored forward output; the row term sum(P * dP),
+    which equals rowsum(dO * O) for the exact O, is then taken as
+    rowsum(dO * out) -- the form a backward pass that receives O as an input
+    computes (so a rounded stored O enters as it does there)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    dO = np.asarray(dO, np.float64)
+    N, D = q.shape
+    bounds = block_bounds(N, Bs)
+    dQ = np.zeros_like(q)
+    dK = np.zeros_like(k)
+    dV = np.zeros_like(v)
+    for i, (a, b) in enumerate(bounds):
+        sel = [int(c) for c in col[int(row_ptr[i]):int(row_ptr[i + 1])]]
+        if not sel:
+            continue
+        keys = np.concatenate([np.arange(*bounds[j]) for j in sel])
+        logits = scale * (q[a:b] @ k[keys].T)
+        e = np.exp(logits - logits.max(axis=1, keepdims=True))
+        P = e / e.sum(axis=1, keepdims=True)
+        dP = dO[a:b] @ v[keys].T
+        if out is None:
+            delta = (P * dP).sum(axis=1, keepdims=True)
+        else:
+            delta = (dO[a:b] * np.asarray(out, np.float64)[a:b]).sum(axis=1, keepdims=True)
+        dS = P * (dP - delta)
+        dQ[a:b] = scale * (dS @ k[keys])
+        np.add.at(dK, keys, scale * (dS.T @ q[a:b]))
+        np.add.at(dV, keys, P.T @ dO[a:b])
+    return dQ, dK, dV
+
+
 def block_mass(lse, blk_lse, row_ptr, N: int, Bs: int) -> np.ndarray:
     """M [nnz]: for slot s of row i, mean_{t in B_i} exp(blk_lse[s,t] - lse_t)."""
     lse = np.asarray(lse, np.float64)

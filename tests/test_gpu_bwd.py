@@ -1,0 +1,82 @@
+"""Backward of the block-sparse attention on the GPU against the fp64
+oracle's chain rule, for the pipeline's own masks and for a hand-built mask
+with an empty row and a key block nobody selects.  The oracle takes the row
+term from the same stored forward output O that the kernel receives.
+
+Gates (per tensor, relative to its largest reference value m):
+fp32 |err| <= 1e-4 m; bf16 |err| <= |ref| / 128 + 2e-3 m (bf16 rounding of
+the stored gradients plus fp32 accumulation)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_pool_b200 import ops, synth
+from oracle import dsa_oracle as O
+from test_gpu_parity import head_csr, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_grads(q, k, v, dO, block, scale, rp, col, grads, out):
+    B, H, N, D = q.shape
+    nB = ops.n_blocks(N, block)
+    rp_c, col_c = rp.cpu().numpy().astype(np.int64), col.cpu().numpy().astype(np.int64)
+    got = [np64(g) for g in grads]
+    for bh in range(B * H):
+        b, h = divmod(bh, H)
+        hrp, hcol, _ = head_csr(rp_c, col_c, bh, nB)
+        ref = O.sparse_attention_backward_head(np64(q[b, h]), np64(k[b, h]), np64(v[b, h]),
+                                               np64(dO[b, h]), block, scale, hrp, hcol,
+                                               out=np64(out[b, h]))
+        for name, g, r in zip("qkv", got, ref):
+            m = max(np.abs(r).max(), 1e-30)
+            err = np.abs(g[b, h] - r)
+            if q.dtype == torch.float32:
+                assert err.max() <= 1e-4 * m, (name, bh, err.max(), m)
+            else:
+                assert np.all(err <= np.abs(r) / 128 + 2e-3 * m), (name, bh, err.max(), m)
+
+
+@pytest.mark.parametrize("w", [synth.TINY, synth.SMALL], ids=lambda w: w.name)
+def test_backward_on_pipeline_mask(w):
+    q, k, v = (t.cuda() for t in synth.make_qkv(w, 17))
+    scale = 1.0 / math.sqrt(w.head_dim)
+    sa = ops.sparse_attention(q, k, v, w.p[0], block=w.block, scale=scale)
+    g = torch.Generator().manual_seed(3)
+    dO = torch.randn(q.shape, generator=g).to(q.dtype).cuda()
+    grads = ops.attn_bwd(q, k, v, sa.out, dO, sa.lse, sa.row_ptr, sa.col_idx, w.block, scale)
+    ops.device_status()
+    nnz = int(sa.row_ptr[-1])
+    _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), w.block, scale, sa.row_ptr,
+                 sa.col_idx[:nnz], grads, sa.out.cpu())
+
+
+def test_backward_empty_row_unselected_block_and_repeatability():
+    w = synth.SMALL
+    q, k, v = (t.cuda() for t in synth.make_qkv(w, 19))
+    B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+    nB = w.n_blocks
+    scale = 1.0 / math.sqrt(D)
+    rows = []
+    for bh in range(B * H):
+        for i in range(nB):
+            if i == 3:
+                rows.append([])                                  # an empty row
+            else:
+                rows.append(sorted({i, (i + 1) % nB, 0} - {5}))  # key block 5: never selected
+    rp = torch.tensor(np.concatenate([[0], np.cumsum([len(r) for r in rows])]), dtype=torch.int32)
+    col = torch.tensor(np.concatenate([np.array(r, dtype=np.int64) for r in rows]), dtype=torch.int32)
+    rpg, colg = rp.cuda(), col.cuda()
+    out, lse, _ = ops.attn_fwd(q, k, v, rpg, colg, blk, scale)
+    dO = torch.randn(q.shape, generator=torch.Generator().manual_seed(8)).to(q.dtype).cuda()
+    g1 = ops.attn_bwd(q, k, v, out, dO, lse, rpg, colg, blk, scale)
+    g2 = ops.attn_bwd(q, k, v, out, dO, lse, rpg, colg, blk, scale)
+    ops.device_status()
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+    dq, dk, dv = (t.cpu() for t in g1)
+    assert torch.all(dq[:, :, 3 * blk:4 * blk] == 0)
+    assert torch.all(dk[:, :, 5 * blk:6 * blk] == 0) and torch.all(dv[:, :, 5 * blk:6 * blk] == 0)
+    _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), blk, scale, rp, col, g1, out.cpu())

@@ -412,3 +412,59 @@ def test_hier_probs_block_constant_closed_form():
     s = 0.7 * qv @ kv.T
     e = n[None, :] * np.exp(s)
     np.testing.assert_allclose(P, e / e.sum(1, keepdims=True), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- backward ----
+
+def test_backward_all_blocks_equals_autograd_of_dense_attention():
+    torch = pytest.importorskip("torch")
+    N, Bs, D, scale = 200, 64, 8, 0.37
+    q, k, v = _qkv(N, D, 31, scale=1.1)
+    dO = np.random.default_rng(32).normal(size=(N, D))
+    nB = 4
+    rp, col = _all_blocks(nB)
+    dQ, dK, dV = O.sparse_attention_backward_head(q, k, v, dO, Bs, scale, rp, col)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    out = torch.softmax(scale * tq @ tk.T, dim=1) @ tv
+    out.backward(torch.tensor(dO))
+    np.testing.assert_allclose(dQ, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dV, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_delta_from_stored_output_matches_exact_form():
+    # sum(P * dP) per row equals rowsum(dO * O) for the exact O
+    N, Bs, D, scale = 96, 32, 5, 0.5
+    q, k, v = _qkv(N, D, 51, scale=1.0)
+    dO = np.random.default_rng(52).normal(size=(N, D))
+    rp = np.array([0, 2, 3, 5])
+    col = np.array([0, 2, 1, 0, 1])
+    out, _, _ = O.sparse_attention_head(q, k, v, Bs, scale, rp, col)
+    a = O.sparse_attention_backward_head(q, k, v, dO, Bs, scale, rp, col)
+    b = O.sparse_attention_backward_head(q, k, v, dO, Bs, scale, rp, col, out=out)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=1e-11, atol=1e-12)
+
+
+def test_backward_masked_matches_finite_differences():
+    N, Bs, D, scale = 40, 16, 3, 0.6
+    q, k, v = _qkv(N, D, 41, scale=1.0)
+    dO = np.random.default_rng(42).normal(size=(N, D))
+    rp = np.array([0, 2, 3, 3])          # row 0: blocks 0, 2; row 1: block 1; row 2: empty
+    col = np.array([2, 0, 1])
+    dQ, dK, dV = O.sparse_attention_backward_head(q, k, v, dO, Bs, scale, rp, col)
+
+    def loss(qq, kk, vv):
+        out, _, _ = O.sparse_attention_head(qq, kk, vv, Bs, scale, rp, col)
+        return float((out * dO).sum())
+    h = 1e-6
+    for name, x, g in (("q", q, dQ), ("k", k, dK), ("v", v, dV)):
+        for (r, c) in [(0, 0), (5, 2), (17, 1), (33, 0), (39, 2)]:
+            xp, xm = x.copy(), x.copy()
+            xp[r, c] += h
+            xm[r, c] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - g[r, c]) <= 1e-6 * max(1.0, abs(fd)), (name, r, c, fd, g[r, c])
+    assert np.all(dQ[32:] == 0)          # empty row: no gradient
