@@ -69,6 +69,10 @@ def parse_args():
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the bench line: one JSON line per point of the "
                          "p-sweep, reduced search, HunyuanVideo schedule and CogVideoX runs")
+    ap.add_argument("--profile-rows", action="store_true",
+                    help="instead of the bench line: run the kernels of the step policy, "
+                         "token reordering, two-level estimate and backward once each on "
+                         "a moderate case (for an ncu launch list)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -502,6 +506,46 @@ def gsrs_run(timed):
             "run_tflops": flops / (t_sparse * 1e-3) / 1e12}
     print(json.dumps(line), flush=True)
 
+def profile_rows():
+    """One pass of each widening row's calls, sized for an ncu capture: the
+    Wan2.1-like grid with 8 heads (Q, K, V 155 MB each, above L2) for the
+    token reordering, the two-level estimate and a search step on exact
+    block masses; one head for the backward (its kernels run ~0.1 s)."""
+    import dataclasses
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = dataclasses.replace(synth.WAN21, heads=8)
+    B, H, N, D, blk = w.batch, w.heads, w.N, w.head_dim, w.block
+    scale = 1.0 / math.sqrt(D)
+    q, k, v = synth.make_qkv(w, 0, device="cuda")
+    # token reordering: gather Q into curve order, scatter it back
+    order = ops.HilbertOrder(w.T, w.Hg, w.W, w.n_prefix, device=dev)
+    qh = order.gather(q)
+    back = order.scatter(qh)
+    # two-level estimate (sub 2)
+    ops.pool_score_hier(q, k, blk, 2, scale)
+    # a search step on exact block masses: attention over a p = 0.95 mask,
+    # its masses as dense rows, Top-p 0.9 within it
+    sa = ops.sparse_attention(q, k, v, 0.95, block=blk, scale=scale)
+    nnz = int(sa.row_ptr[-1])
+    P = ops.mass_to_probs(sa.row_ptr, sa.col_idx, sa.mass, w.n_blocks)
+    rp2, _ = ops.select_topp(P, 0.9, cand=(sa.row_ptr, sa.col_idx))
+    ops.device_status(dev)
+    ok_perm = bool(torch.equal(back, q))
+    del q, k, v, qh, back, sa, P
+    # backward on one head at p = 0.9
+    w1 = dataclasses.replace(synth.WAN21, heads=1)
+    q, k, v = synth.make_qkv(w1, 0, device="cuda")
+    s1 = ops.sparse_attention(q, k, v, 0.9, block=blk, scale=scale)
+    dO = torch.randn(q.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(1)).to(q.dtype)
+    ops.attn_bwd(q, k, v, s1.out, dO, s1.lse, s1.row_ptr, s1.col_idx, blk, scale)
+    ops.device_status(dev)
+    torch.cuda.synchronize(dev)
+    print(json.dumps({"profile_rows": "wan2.1-like", "heads": H, "scatter_inverts_gather": ok_perm,
+                      "search_step_mask_nnz": nnz, "reselected_nnz": int(rp2[-1]),
+                      "bwd_heads": 1, "bwd_nnz": int(s1.row_ptr[-1])}), flush=True)
+
+
 # ---------------------------------------------------------------- GPU bench --
 
 def main():
@@ -512,6 +556,9 @@ def main():
         return
     if args.sweep:
         sweep(args)
+        return
+    if args.profile_rows:
+        profile_rows()
         return
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
