@@ -433,10 +433,13 @@ def sweep(args):
 
 
 def backward_point(timed):
-    """Backward of the attention (exact fp32 on CUDA cores) on the Wan2.1-like
-    grid with 8 heads at p = 0.9.  Algorithmic FLOPs: the five contractions
-    (Q K^T, dO V^T, dS K, dS^T Q, P^T dO) = 2.5 x the forward's executed
-    FLOPs; this kernel also recomputes Q K^T and dO V^T in its dK/dV pass."""
+    """Backward of the attention on the Wan2.1-like grid with 8 heads at
+    p = 0.9 (bf16, blocks of 128: the tcgen05 kernels).  Algorithmic FLOPs:
+    the five contractions (Q K^T, dO V^T, dS K, dS^T Q, P^T dO) = 2.5 x the
+    forward's executed FLOPs.  Executed on the tensor cores: 5 x the
+    forward's -- Q K^T and dO V^T are computed on both sides (dq and dkdv
+    kernels), and each gradient product runs twice (bf16 hi and lo terms of
+    P and dS)."""
     import dataclasses
     dev = torch.device("cuda", 0)
     w = dataclasses.replace(synth.WAN21, heads=8)
@@ -450,11 +453,15 @@ def backward_point(timed):
                              workspace=ws)
     f()
     ops.device_status(dev)
-    t = timed(f, 2)
+    t = timed(f, 3)
     fwd, nnz = executed_flops(sa.row_ptr, sa.col_idx, N, blk, D, w.n_blocks)
-    line = {"sweep": "backward (exact fp32 on CUDA cores), wan2.1-like 8 heads", "p": 0.9,
+    peak = measured_peaks()["bf16_sustained"]
+    line = {"sweep": "backward (tcgen05, P and dS as bf16 hi + lo), wan2.1-like 8 heads", "p": 0.9,
             "nnz_blocks": nnz, "bwd_ms": t, "algorithmic_tflop": 2.5 * fwd / 1e12,
-            "bwd_tflops": 2.5 * fwd / (t * 1e-3) / 1e12, "bound": "fp32 CUDA cores"}
+            "bwd_tflops": 2.5 * fwd / (t * 1e-3) / 1e12,
+            "executed_tensor_tflops": 5 * fwd / (t * 1e-3) / 1e12,
+            "frac_of_bf16_sustained_peak_executed": (5 * fwd / (t * 1e-3) / 1e12 / peak) if peak else None,
+            "bound": "tensor (element-wise P, dS between the products)"}
     print(json.dumps(line), flush=True)
 
 

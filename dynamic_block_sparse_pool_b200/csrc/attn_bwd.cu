@@ -372,6 +372,10 @@ cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const v
                                                       static_cast<const float*>(dout), tok, delta);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // bf16 with blocks of 128: the tensor-core kernels; otherwise exact fp32 on CUDA cores
+  if (bf16 && block == 128)
+    return launch_attn_bwd_sm100(q, k, v, dout, lse, delta, BH, N, D, scale, row_ptr, col_idx,
+                                 t_row_ptr, t_col, dq, dk, dv, err, s);
   if (bf16)
     return launch_grads_t<__nv_bfloat16>(D, block, q, k, v, dout, lse, delta, BH, N, nB, scale,
                                          row_ptr, col_idx, t_row_ptr, t_col, dq, dk, dv, s);

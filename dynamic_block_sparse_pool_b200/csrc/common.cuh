@@ -75,6 +75,13 @@ cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const v
                             const int32_t* col_idx, void* dq, void* dk, void* dv,
                             uint32_t* bitmap, int32_t* counts, int32_t* t_row_ptr,
                             int32_t* t_col, float* delta, unsigned* err, cudaStream_t s);
+// dQ, dK, dV on tcgen05 (bf16, blocks of 128): after the mask transpose and
+// the row term delta of launch_attn_bwd.
+cudaError_t launch_attn_bwd_sm100(const void* q, const void* k, const void* v, const void* dout,
+                                  const float* lse, const float* delta, int BH, int N, int D,
+                                  float scale, const int32_t* row_ptr, const int32_t* col_idx,
+                                  const int32_t* t_row_ptr, const int32_t* t_col, void* dq, void* dk,
+                                  void* dv, unsigned* err, cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

@@ -1,7 +1,10 @@
 """Backward of the block-sparse attention on the GPU against the fp64
-oracle's chain rule, for the pipeline's own masks and for a hand-built mask
-with an empty row and a key block nobody selects.  The oracle takes the row
-term from the same stored forward output O that the kernel receives.
+oracle's chain rule, for the pipeline's own masks, for random fixed masks
+(ragged tails, empty rows) and for a hand-built mask with an empty row and a
+key block nobody selects.  The oracle takes the row term from the same stored
+forward output O that the kernel receives.  bf16 with blocks of 128 runs on
+the tensor-core kernels (P and dS as bf16 hi + lo terms), fp32 and blocks of
+64 on the fp32 CUDA-core kernels; both meet the same gates.
 
 Gates (per tensor, relative to its largest reference value m):
 fp32 |err| <= 1e-4 m; bf16 |err| <= |ref| / 128 + 2e-3 m (bf16 rounding of
@@ -51,6 +54,24 @@ def test_backward_on_pipeline_mask(w):
     nnz = int(sa.row_ptr[-1])
     _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), w.block, scale, sa.row_ptr,
                  sa.col_idx[:nnz], grads, sa.out.cpu())
+
+
+@pytest.mark.parametrize("name,B,H,N,D,block,density", [
+    ("tc_d128_ragged", 1, 2, 1000, 128, 128, 0.5),
+    ("tc_d128_dense_rows", 1, 1, 128 * 9 + 40, 128, 128, 1.0),
+    ("tc_d64_long_rows", 2, 1, 128 * 12 + 5, 64, 128, 0.8),
+    ("simt_bf16_block64", 1, 2, 300, 64, 64, 0.5),
+])
+def test_backward_fixed_mask(name, B, H, N, D, block, density):
+    q, k, v = (t.cuda() for t in synth.random_qkv(B, H, N, D, torch.bfloat16, seed=41))
+    nB = ops.n_blocks(N, block)
+    rp, col = synth.random_csr(B * H * nB, nB, density, seed=5)
+    scale = 1.0 / math.sqrt(D)
+    out, lse, _ = ops.attn_fwd(q, k, v, rp.cuda(), col.cuda(), block, scale)
+    dO = torch.randn(q.shape, generator=torch.Generator().manual_seed(6)).to(q.dtype).cuda()
+    grads = ops.attn_bwd(q, k, v, out, dO, lse, rp.cuda(), col.cuda(), block, scale)
+    ops.device_status()
+    _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), block, scale, rp, col, grads, out.cpu())
 
 
 def test_backward_empty_row_unselected_block_and_repeatability():
