@@ -517,7 +517,7 @@ def profile_rows():
     """One pass of each widening row's calls, sized for an ncu capture: the
     Wan2.1-like grid with 8 heads (Q, K, V 155 MB each, above L2) for the
     token reordering, the two-level estimate and a search step on exact
-    block masses; one head for the backward (its kernels run ~0.1 s)."""
+    block masses; one head for the backward."""
     import dataclasses
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
