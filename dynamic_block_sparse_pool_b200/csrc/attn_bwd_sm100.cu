@@ -28,6 +28,13 @@
 // the dP^T chunk.  An MMA K-step of 16 elements reads 8 packed columns, so
 // step kk takes its A operand at column 32 (kk / 2) + 8 (kk % 2) (+16 for lo).
 //
+// Each block's S-type products run as two halves of 64 columns with their own
+// barriers: the element-wise warps start on the first half while the second
+// is computed, and the MMA warp issues the first half's gradient product and
+// the next block's first half while they work on the second, so the tensor
+// pipe and the element-wise pass overlap within the one S/dP buffer that
+// tensor memory leaves room for.
+//
 // Warps 0-3: element-wise (thread = tensor-memory lane = row of the block);
 // warp 4: MMA issuer (one thread) and tensor-memory allocation; warp 5: TMA
 // loader (one thread).  Tensor memory: S 0-127, dP 128-255, then the fp32
@@ -50,7 +57,8 @@ constexpr uint32_t kColS = 0, kColP = 128, kColG = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // barriers (8 bytes each)
-enum : int { kBarFixed = 0, kBarRing = 1, kBarFree = 3, kBarS = 5, kBarP = 6, kNumBars = 7 };
+// (kBarS, kBarP: one per half of the block's columns)
+enum : int { kBarFixed = 0, kBarRing = 1, kBarFree = 3, kBarS = 5, kBarP = 7, kNumBars = 9 };
 
 template <int D>
 struct BwdSmem {
@@ -100,25 +108,31 @@ __device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint3
   lo = pack_bf16(a - __low2float(h), b - __high2float(h));
 }
 
-// S-type product: D[tmem] = A B^T, both [128 x D] tiles K-major
+// S-type product for half h of the block's columns: D[tmem, 64 columns] =
+// A B_h^T, A a [128 x D] tile and B_h rows 64h .. 64h + 63 of another, both
+// K-major (64 rows of 128 bytes per 64-column sub-tile: 8192 bytes on).
 template <int D>
-__device__ __forceinline__ void mma_rows(uint32_t d, uint64_t a0, uint64_t b0) {
-  constexpr uint32_t kIdesc = idesc_bf16_f32(BB, BB, false);
-  mma_ss(d, a0 + kstep<D>(0), b0 + kstep<D>(0), kIdesc, 0u);
+__device__ __forceinline__ void mma_rows_half(uint32_t d, uint64_t a0, uint64_t b0, int h) {
+  constexpr uint32_t kIdesc = idesc_bf16_f32(BB, BB / 2, false);
+  const uint64_t bh = b0 + (uint64_t)((h * (BB / 2) * 128) >> 4);
+  mma_ss(d, a0 + kstep<D>(0), bh + kstep<D>(0), kIdesc, 0u);
 #pragma unroll
-  for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, a0 + kstep<D>(kk), b0 + kstep<D>(kk), kIdesc);
+  for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, a0 + kstep<D>(kk), bh + kstep<D>(kk), kIdesc);
 }
 
-// gradient product: D[tmem] (+)= (hi + lo)[tmem, 128 x 128 packed as above] B,
-// B a [128 x D] tile read MN-major (its rows are the K dimension)
+// gradient product over half h of the K dimension: D[tmem] (+)= (hi + lo)
+// [tmem, rows x K steps 4h .. 4h + 3, packed as above] B, B a [128 x D] tile
+// read MN-major (its rows are the K dimension)
 template <int D>
-__device__ __forceinline__ void mma_grad(uint32_t d, uint32_t a, uint64_t b0, bool accumulate) {
+__device__ __forceinline__ void mma_grad_half(uint32_t d, uint32_t a, uint64_t b0, int h,
+                                              bool accumulate) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(BB, D, true);
 #pragma unroll
-  for (int kk = 0; kk < BB / 16; ++kk) {
+  for (int q = 0; q < 4; ++q) {
+    const int kk = 4 * h + q;
     const uint32_t ah = a + 32u * (uint32_t)(kk >> 1) + 8u * (uint32_t)(kk & 1);
     const uint64_t b = b0 + (uint64_t)((kk * 2048) >> 4);
-    if (kk == 0 && !accumulate)
+    if (q == 0 && !accumulate)
       mma_ts(d, ah, b, kIdesc, 0u);
     else
       mma_ts_acc(d, ah, b, kIdesc);
@@ -172,7 +186,7 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
   if (warp == kMmaWarp) {
     if (lane == 0) {
-      for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), i == kBarP ? 4u : 1u);
+      for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == kBarP || i == kBarP + 1) ? 4u : 1u);
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -232,31 +246,38 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const uint64_t dKk = smem_desc_sw128(sK, 16, 1024), dVk = smem_desc_sw128(sV, 16, 1024);
       const uint64_t dKm = smem_desc_sw128(sK, L::kSub, 1024);
       bool ok = warp_all(mbar_wait(bar(kBarFixed), 0u));
-      auto issue_sdp = [&](int it) {
+      // S and dP of half h (keys 64h .. 64h + 63) of block it
+      auto issue_half = [&](int it, int h) {
         const int s = it & 1;
-        if (!(ok = ok && warp_all(mbar_wait(bar(kBarRing + s), (uint32_t)(it >> 1) & 1u)))) return;
+        if (h == 0 && !(ok = ok && warp_all(mbar_wait(bar(kBarRing + s), (uint32_t)(it >> 1) & 1u))))
+          return;
         tc_fence_after();
         if (leader) {
           const uint64_t off = (uint64_t)((s * kTileBytes) >> 4);
-          mma_rows<D>(tmem + kColS, dQk, dKk + off);
-          mma_rows<D>(tmem + kColP, dOk, dVk + off);
-          mma_commit(bar(kBarS));
+          mma_rows_half<D>(tmem + kColS + 64 * h, dQk, dKk + off, h);
+          mma_rows_half<D>(tmem + kColP + 64 * h, dOk, dVk + off, h);
+          mma_commit(bar(kBarS + h));
         }
         __syncwarp();
       };
-      issue_sdp(0);
+      issue_half(0, 0);
+      if (ok) issue_half(0, 1);
       for (int it = 0; it < n && ok; ++it) {
         const int s = it & 1;
-        if (!(ok = warp_all(mbar_wait(bar(kBarP), (uint32_t)it & 1u)))) break;
-        tc_fence_after();
-        if (leader) {
-          mma_grad<D>(tmem + kColG, tmem + kColS, dKm + (uint64_t)((s * kTileBytes) >> 4), it > 0);
-          mma_commit(bar(kBarFree + s));
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!(ok = warp_all(mbar_wait(bar(kBarP + h), (uint32_t)it & 1u)))) break;
+          tc_fence_after();
+          if (leader) {
+            mma_grad_half<D>(tmem + kColG, tmem + kColS, dKm + (uint64_t)((s * kTileBytes) >> 4), h,
+                             it > 0 || h > 0);
+            if (h == 1) mma_commit(bar(kBarFree + s));
+          }
+          __syncwarp();
+          // half h of block it + 1 overwrites half h's dS columns only after
+          // dQ has read them (the MMAs of one thread run in order), while the
+          // element-wise warps work on the other half
+          if (it + 1 < n) issue_half(it + 1, h);
         }
-        __syncwarp();
-        // S(it + 1) overwrites the dS columns only after dQ(it) has read
-        // them: the MMAs of one thread run in order
-        if (it + 1 < n) issue_sdp(it + 1);
       }
       if (!ok && leader) {
         *abort_flag = 1;
@@ -272,36 +293,39 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const float lse2 = valid ? lse[tok] * kLog2e : INFINITY;
     const float dl = valid ? delta[tok] : 0.f;
     bool failed = false;
-    for (int it = 0; it < n; ++it) {
+    for (int it = 0; it < n && !failed; ++it) {
       const int kvv = col_idx[s0 + it] == nB - 1 ? kv_last : BB;  // keys in the block
-      if (!warp_all(mbar_wait(bar(kBarS), (uint32_t)it & 1u))) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BB / 32; ++c) {
-        uint32_t sv[32], pv[32];
-        tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
-        tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
-        tmem_wait_ld_regs(sv);
-        tmem_wait_ld_regs(pv);
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const int key = 32 * c + 2 * m;
-          const float p0 = key < kvv ? exp2_approx(__uint_as_float(sv[2 * m]) * scale_log2 - lse2) : 0.f;
-          const float p1 = key + 1 < kvv ? exp2_approx(__uint_as_float(sv[2 * m + 1]) * scale_log2 - lse2) : 0.f;
-          split_pair(p0 * (__uint_as_float(pv[2 * m]) - dl), p1 * (__uint_as_float(pv[2 * m + 1]) - dl),
-                     hi[m], lo[m]);
+      for (int h = 0; h < 2; ++h) {
+        if (!warp_all(mbar_wait(bar(kBarS + h), (uint32_t)it & 1u))) {
+          failed = true;
+          break;
         }
-        tmem_st16(tmem + lane_off + kColS + 32 * c, hi);
-        tmem_st16(tmem + lane_off + kColS + 32 * c + 16, lo);
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * h + cc;
+          uint32_t sv[32], pv[32];
+          tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
+          tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
+          tmem_wait_ld_regs(sv);
+          tmem_wait_ld_regs(pv);
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const int key = 32 * c + 2 * m;
+            const float p0 = key < kvv ? exp2_approx(__uint_as_float(sv[2 * m]) * scale_log2 - lse2) : 0.f;
+            const float p1 = key + 1 < kvv ? exp2_approx(__uint_as_float(sv[2 * m + 1]) * scale_log2 - lse2) : 0.f;
+            split_pair(p0 * (__uint_as_float(pv[2 * m]) - dl), p1 * (__uint_as_float(pv[2 * m + 1]) - dl),
+                       hi[m], lo[m]);
+          }
+          tmem_st16(tmem + lane_off + kColS + 32 * c, hi);
+          tmem_st16(tmem + lane_off + kColS + 32 * c + 16, lo);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarP + h));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarP));
     }
     __nv_bfloat16* drow = dq + tok * D;
     if (failed) {
@@ -369,7 +393,7 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 
   if (warp == kMmaWarp) {
     if (lane == 0) {
-      for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), i == kBarP ? 4u : 1u);
+      for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == kBarP || i == kBarP + 1) ? 4u : 1u);
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -422,31 +446,36 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       const uint64_t dQk = smem_desc_sw128(sQ, 16, 1024), dOk = smem_desc_sw128(sO, 16, 1024);
       const uint64_t dQm = smem_desc_sw128(sQ, L::kSub, 1024), dOm = smem_desc_sw128(sO, L::kSub, 1024);
       bool ok = warp_all(mbar_wait(bar(kBarFixed), 0u));
-      auto issue_sdp = [&](int it) {
+      // S^T and dP^T of half h (queries 64h .. 64h + 63) of block it
+      auto issue_half = [&](int it, int h) {
         const int s = it & 1;
-        if (!(ok = ok && warp_all(mbar_wait(bar(kBarRing + s), (uint32_t)(it >> 1) & 1u)))) return;
+        if (h == 0 && !(ok = ok && warp_all(mbar_wait(bar(kBarRing + s), (uint32_t)(it >> 1) & 1u))))
+          return;
         tc_fence_after();
         if (leader) {
           const uint64_t off = (uint64_t)((s * kTileBytes) >> 4);
-          mma_rows<D>(tmem + kColS, dKk, dQk + off);  // S^T = K Q^T
-          mma_rows<D>(tmem + kColP, dVk, dOk + off);  // dP^T = V dO^T
-          mma_commit(bar(kBarS));
+          mma_rows_half<D>(tmem + kColS + 64 * h, dKk, dQk + off, h);  // S^T = K Q^T
+          mma_rows_half<D>(tmem + kColP + 64 * h, dVk, dOk + off, h);  // dP^T = V dO^T
+          mma_commit(bar(kBarS + h));
         }
         __syncwarp();
       };
-      issue_sdp(0);
+      issue_half(0, 0);
+      if (ok) issue_half(0, 1);
       for (int it = 0; it < n && ok; ++it) {
         const int s = it & 1;
-        if (!(ok = warp_all(mbar_wait(bar(kBarP), (uint32_t)it & 1u)))) break;
-        tc_fence_after();
-        if (leader) {
-          const uint64_t off = (uint64_t)((s * kTileBytes) >> 4);
-          mma_grad<D>(tmem + kColV, tmem + kColS, dOm + off, it > 0);  // dV += P^T dO
-          mma_grad<D>(tmem + kColK, tmem + kColP, dQm + off, it > 0);  // dK += dS^T Q
-          mma_commit(bar(kBarFree + s));
+        const uint64_t off = (uint64_t)((s * kTileBytes) >> 4);
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!(ok = warp_all(mbar_wait(bar(kBarP + h), (uint32_t)it & 1u)))) break;
+          tc_fence_after();
+          if (leader) {
+            mma_grad_half<D>(tmem + kColV, tmem + kColS, dOm + off, h, it > 0 || h > 0);  // dV += P^T dO
+            mma_grad_half<D>(tmem + kColK, tmem + kColP, dQm + off, h, it > 0 || h > 0);  // dK += dS^T Q
+            if (h == 1) mma_commit(bar(kBarFree + s));
+          }
+          __syncwarp();
+          if (it + 1 < n) issue_half(it + 1, h);
         }
-        __syncwarp();
-        if (it + 1 < n) issue_sdp(it + 1);
       }
       if (!ok && leader) {
         *abort_flag = 1;
@@ -468,42 +497,46 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       const size_t tok = (size_t)bh * N + q0 + row;
       lse2[row] = row < qlen ? lse[tok] * kLog2e : INFINITY;
       dls[row] = row < qlen ? delta[tok] : 0.f;
-      // One barrier of the four warps serves two ends: it publishes the
-      // vectors just written (the other buffer was last read before it),
-      // and it makes a timed-out wait a decision of all four warps, so none
-      // is left alone at the next iteration's barrier.
-      const bool late = !warp_all(mbar_wait(bar(kBarS), (uint32_t)it & 1u));
-      if (named_bar_or(1, 128, late)) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BB / 32; ++c) {
-        uint32_t sv[32], pv[32];
-        tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
-        tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
-        tmem_wait_ld_regs(sv);
-        tmem_wait_ld_regs(pv);
-        uint32_t ph[16], pl[16], dh[16], dl[16];
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const int qq = 32 * c + 2 * m;
-          const float p0 = exp2_approx(__uint_as_float(sv[2 * m]) * scale_log2 - lse2[qq]);
-          const float p1 = exp2_approx(__uint_as_float(sv[2 * m + 1]) * scale_log2 - lse2[qq + 1]);
-          split_pair(p0, p1, ph[m], pl[m]);
-          split_pair(p0 * (__uint_as_float(pv[2 * m]) - dls[qq]),
-                     p1 * (__uint_as_float(pv[2 * m + 1]) - dls[qq + 1]), dh[m], dl[m]);
+      // A barrier of the four warps at each half serves two ends: it makes a
+      // timed-out wait a decision of all four warps, so none is left alone at
+      // a later barrier, and the first one publishes the vectors just written
+      // (the other buffer was last read before it).
+      for (int h = 0; h < 2; ++h) {
+        const bool late = !warp_all(mbar_wait(bar(kBarS + h), (uint32_t)it & 1u));
+        if (named_bar_or(1, 128, late)) {
+          failed = true;
+          break;
         }
-        tmem_st16(tmem + lane_off + kColS + 32 * c, ph);
-        tmem_st16(tmem + lane_off + kColS + 32 * c + 16, pl);
-        tmem_st16(tmem + lane_off + kColP + 32 * c, dh);
-        tmem_st16(tmem + lane_off + kColP + 32 * c + 16, dl);
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * h + cc;
+          uint32_t sv[32], pv[32];
+          tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
+          tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
+          tmem_wait_ld_regs(sv);
+          tmem_wait_ld_regs(pv);
+          uint32_t ph[16], pl[16], dh[16], dl[16];
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const int qq = 32 * c + 2 * m;
+            const float p0 = exp2_approx(__uint_as_float(sv[2 * m]) * scale_log2 - lse2[qq]);
+            const float p1 = exp2_approx(__uint_as_float(sv[2 * m + 1]) * scale_log2 - lse2[qq + 1]);
+            split_pair(p0, p1, ph[m], pl[m]);
+            split_pair(p0 * (__uint_as_float(pv[2 * m]) - dls[qq]),
+                       p1 * (__uint_as_float(pv[2 * m + 1]) - dls[qq + 1]), dh[m], dl[m]);
+          }
+          tmem_st16(tmem + lane_off + kColS + 32 * c, ph);
+          tmem_st16(tmem + lane_off + kColS + 32 * c + 16, pl);
+          tmem_st16(tmem + lane_off + kColP + 32 * c, dh);
+          tmem_st16(tmem + lane_off + kColP + 32 * c + 16, dl);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarP + h));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarP));
+      if (failed) break;
     }
     const bool valid = row < klen;
     const size_t ktok = (size_t)bh * N + k0 + row;
