@@ -68,7 +68,7 @@ struct BwdSmem {
   static constexpr int kFixB = kTile;
   static constexpr int kRingA = 2 * kTile;   // ring of the first streamed tile, 2 stages
   static constexpr int kRingB = 4 * kTile;   // ring of the second streamed tile
-  static constexpr int kVec = 6 * kTile;     // float [2][2][128]: lse2, delta of the current query block (dkdv)
+  static constexpr int kVec = 6 * kTile;     // float [2][2][128]: -lse2, -delta of the current query block (dkdv)
   static constexpr int kBar = kVec + 2 * 2 * BB * 4;
   static constexpr int kSlot = kBar + 8 * kNumBars;
   static constexpr int kBytes = kSlot + 16;
@@ -290,11 +290,16 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     const bool valid = row < qlen;
     const size_t tok = (size_t)bh * N + q0 + row;
-    const float lse2 = valid ? lse[tok] * kLog2e : INFINITY;
-    const float dl = valid ? delta[tok] : 0.f;
+    // -lse (base 2) and -delta of the row, as packed pairs; rows past N get
+    // -inf, so their P is 0
+    const float nl = valid ? -lse[tok] * kLog2e : -INFINITY;
+    const float nd = valid ? -delta[tok] : 0.f;
+    const uint64_t sc2 = pack_f32x2(scale_log2, scale_log2);
+    const uint64_t nl2 = pack_f32x2(nl, nl), nd2 = pack_f32x2(nd, nd);
     bool failed = false;
     for (int it = 0; it < n && !failed; ++it) {
-      const int kvv = col_idx[s0 + it] == nB - 1 ? kv_last : BB;  // keys in the block
+      // the ragged last key block: keys past N get S = -inf, so P = 0
+      const bool rag = kv_last < BB && col_idx[s0 + it] == nB - 1;
       for (int h = 0; h < 2; ++h) {
         if (!warp_all(mbar_wait(bar(kBarS + h), (uint32_t)it & 1u))) {
           failed = true;
@@ -309,14 +314,21 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
           tmem_wait_ld_regs(sv);
           tmem_wait_ld_regs(pv);
+          if (rag) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              if (32 * c + u >= kv_last) sv[u] = __float_as_uint(-INFINITY);
+          }
           uint32_t hi[16], lo[16];
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            const int key = 32 * c + 2 * m;
-            const float p0 = key < kvv ? exp2_approx(__uint_as_float(sv[2 * m]) * scale_log2 - lse2) : 0.f;
-            const float p1 = key + 1 < kvv ? exp2_approx(__uint_as_float(sv[2 * m + 1]) * scale_log2 - lse2) : 0.f;
-            split_pair(p0 * (__uint_as_float(pv[2 * m]) - dl), p1 * (__uint_as_float(pv[2 * m + 1]) - dl),
-                       hi[m], lo[m]);
+            float t0, t1, g0, g1;
+            unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[2 * m]), __uint_as_float(sv[2 * m + 1])),
+                                   sc2, nl2), t0, t1);
+            const uint64_t p2 = pack_f32x2(exp2_approx(t0), exp2_approx(t1));
+            const uint64_t d2 = add_f32x2(pack_f32x2(__uint_as_float(pv[2 * m]), __uint_as_float(pv[2 * m + 1])), nd2);
+            unpack_f32x2(mul_f32x2(p2, d2), g0, g1);
+            split_pair(g0, g1, hi[m], lo[m]);
           }
           tmem_st16(tmem + lane_off + kColS + 32 * c, hi);
           tmem_st16(tmem + lane_off + kColS + 32 * c + 16, lo);
@@ -380,7 +392,7 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   }
   const uint32_t sK = base + L::kFixA, sV = base + L::kFixB;    // K, V of the key block
   const uint32_t sQ = base + L::kRingA, sO = base + L::kRingB;  // Q, dO of the query blocks
-  float* vec = reinterpret_cast<float*>(smem + L::kVec);        // [buf][lse2 | delta][128]
+  float* vec = reinterpret_cast<float*>(smem + L::kVec);        // [buf][-lse2 | -delta][128]
   const uint32_t bars = base + L::kBar;
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlot);
@@ -487,16 +499,18 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     // thread = key row of the block; columns = the query block's queries
     const int row = 32 * warp + lane;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint64_t sc2 = pack_f32x2(scale_log2, scale_log2);
     bool failed = false;
     for (int it = 0; it < n; ++it) {
       const int i = t_col[t0 + it];
       const int q0 = i * BB, qlen = min(BB, N - q0);
-      float* lse2 = vec + (it & 1) * 2 * BB;
-      float* dls = lse2 + BB;
-      // this query block's lse (base 2) and delta; queries past N get P = 0
+      float* nl = vec + (it & 1) * 2 * BB;
+      float* nd = nl + BB;
+      // this query block's -lse (base 2) and -delta; queries past N get
+      // -inf, so their P is 0
       const size_t tok = (size_t)bh * N + q0 + row;
-      lse2[row] = row < qlen ? lse[tok] * kLog2e : INFINITY;
-      dls[row] = row < qlen ? delta[tok] : 0.f;
+      nl[row] = row < qlen ? -lse[tok] * kLog2e : -INFINITY;
+      nd[row] = row < qlen ? -delta[tok] : 0.f;
       // A barrier of the four warps at each half serves two ends: it makes a
       // timed-out wait a decision of all four warps, so none is left alone at
       // a later barrier, and the first one publishes the vectors just written
@@ -519,12 +533,16 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
           uint32_t ph[16], pl[16], dh[16], dl[16];
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            const int qq = 32 * c + 2 * m;
-            const float p0 = exp2_approx(__uint_as_float(sv[2 * m]) * scale_log2 - lse2[qq]);
-            const float p1 = exp2_approx(__uint_as_float(sv[2 * m + 1]) * scale_log2 - lse2[qq + 1]);
+            const int qq = 32 * c + 2 * m;  // even: the pairs are 8-byte aligned
+            float t0, t1, g0, g1;
+            unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[2 * m]), __uint_as_float(sv[2 * m + 1])),
+                                   sc2, *reinterpret_cast<const uint64_t*>(nl + qq)), t0, t1);
+            const float p0 = exp2_approx(t0), p1 = exp2_approx(t1);
             split_pair(p0, p1, ph[m], pl[m]);
-            split_pair(p0 * (__uint_as_float(pv[2 * m]) - dls[qq]),
-                       p1 * (__uint_as_float(pv[2 * m + 1]) - dls[qq + 1]), dh[m], dl[m]);
+            const uint64_t d2 = add_f32x2(pack_f32x2(__uint_as_float(pv[2 * m]), __uint_as_float(pv[2 * m + 1])),
+                                          *reinterpret_cast<const uint64_t*>(nd + qq));
+            unpack_f32x2(mul_f32x2(pack_f32x2(p0, p1), d2), g0, g1);
+            split_pair(g0, g1, dh[m], dl[m]);
           }
           tmem_st16(tmem + lane_off + kColS + 32 * c, ph);
           tmem_st16(tmem + lane_off + kColS + 32 * c + 16, pl);
