@@ -161,7 +161,10 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.T
 def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
              dout: torch.Tensor, lse: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
              block: int, scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None):
-    """(dQ, dK, dV) [B, H, N, D] of attn_fwd's O for a fixed mask, given dO."""
+    """(dQ, dK, dV) [B, H, N, D] of attn_fwd's O for a fixed mask, given dO.
+
+    bf16 with block 128 runs on the tensor cores (P and dS as bf16 hi + lo
+    terms); fp32 and block 64 in exact fp32 on CUDA cores."""
     B, H, N, D = _check_qkv(q, k, v)
     for t in (out, dout):
         if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():

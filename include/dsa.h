@@ -205,7 +205,10 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
  *              selected get dK = dV = 0, queries of empty rows dQ = 0.
  *   workspace  >= dsa_workspace_size(DSA_OP_ATTN_BWD, ...) bytes, 16-byte
  *              aligned.
- * Exact fp32 arithmetic on CUDA cores for both dtypes.  Every key block's
+ * Arithmetic: bf16 with block 128 runs on tcgen05 tensor cores with fp32
+ * accumulation, and P and dS enter the gradient products as two bf16 terms
+ * each (hi = bf16(x), lo = bf16(x - hi)), about 2^-17 of each term; fp32,
+ * and block 64, run in exact fp32 on CUDA cores.  Every key block's
  * contributions are summed in ascending query-block order, so the result is
  * the same from run to run.  Errors as for dsa_attn_fwd; a malformed mask
  * sets the device error word.
