@@ -32,6 +32,41 @@ def test_header_declares_the_four_pipeline_calls():
         assert name in syms
 
 
+def declared_prototypes():
+    """name -> (return type, [parameter types]) for every prototype in dsa.h."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for ret, name, params in re.findall(
+            r"^\s*((?:const\s+)?[a-z_0-9]+\s*\**)\s*(dsa_[a-z_]+)\s*\(([^)]*)\)\s*;",
+            text, flags=re.M):
+        params = " ".join(params.split())
+        types = [] if params in ("", "void") else [
+            re.sub(r"\s*\b[A-Za-z_][A-Za-z_0-9]*$", "", p.strip()) for p in params.split(",")]
+        protos[name] = (" ".join(ret.split()), types)
+    return protos
+
+
+def _ctype_of(c):
+    """The ctypes type the binding must use for a C parameter or return type."""
+    c = " ".join(c.replace("*", " * ").split())
+    if c.endswith("*"):
+        return ctypes.c_char_p if c == "const char *" else ctypes.c_void_p
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+            "dsa_dtype": ctypes.c_int, "dsa_status": ctypes.c_int}[c]
+
+
+def test_binding_signatures_match_the_header():
+    # every prototype's argument count and types, and its return type, as the
+    # ctypes binding declares them (a mismatch would pass a wrong value to
+    # the library without any error)
+    protos = declared_prototypes()
+    assert set(protos) == set(_lib.SIGNATURES), set(protos) ^ set(_lib.SIGNATURES)
+    for name, (ret, params) in protos.items():
+        res, args = _lib.SIGNATURES[name]
+        assert res == _ctype_of(ret), (name, ret, res)
+        assert [_ctype_of(t) for t in params] == list(args), (name, params, args)
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
