@@ -87,6 +87,7 @@ def measured_peaks():
             d = json.load(f)
         return dict(bf16_burst=float(d["bf16_tflops"]),
                     bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    sustained_sm_mhz=d.get("clocks_under_load", {}).get("sm_mhz_median"),
                     hbm=float(d["hbm_gbs"]), source="measured")
     return dict(bf16_burst=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
@@ -455,12 +456,13 @@ def backward_point(timed):
     ops.device_status(dev)
     t = timed(f, 3)
     fwd, nnz = executed_flops(sa.row_ptr, sa.col_idx, N, blk, D, w.n_blocks)
-    peak = measured_peaks()["bf16_sustained"]
+    peak = measured_peaks()["bf16_burst"]
     line = {"sweep": "backward (tcgen05, P and dS as bf16 hi + lo), wan2.1-like 8 heads", "p": 0.9,
             "nnz_blocks": nnz, "bwd_ms": t, "algorithmic_tflop": 2.5 * fwd / 1e12,
             "bwd_tflops": 2.5 * fwd / (t * 1e-3) / 1e12,
             "executed_tensor_tflops": 5 * fwd / (t * 1e-3) / 1e12,
-            "frac_of_bf16_sustained_peak_executed": (5 * fwd / (t * 1e-3) / 1e12 / peak) if peak else None,
+            "frac_of_bf16_burst_peak_algorithmic": 2.5 * fwd / (t * 1e-3) / 1e12 / peak,
+            "frac_of_bf16_burst_peak_executed": 5 * fwd / (t * 1e-3) / 1e12 / peak,
             "bound": "tensor (element-wise P, dS between the products)"}
     print(json.dumps(line), flush=True)
 
@@ -644,12 +646,16 @@ def main():
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
     }
     traffic = ATTN_TRAFFIC.get(attn_source_hash())
+    # The denominator is the measured burst cuBLAS bf16 rate: the sustained
+    # figure was taken at a lower median SM clock than this loop runs at, so
+    # it would flatter the fraction; it is reported beside it for context.
     line["roofline"] = {
         "bound": "tensor", "kernel": "attn_fwd_sm100_kernel", "achieved": attn_tflops,
-        "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-        "frac": attn_tflops / peaks["bf16_sustained"],
-        "peak_kind": f"{peaks['source']} bf16 sustained (kernel timed inside multi-second step loop)",
-        "frac_of_burst_peak": attn_tflops / peaks["bf16_burst"],
+        "peak": peaks["bf16_burst"], "unit": "TFLOP/s",
+        "frac": attn_tflops / peaks["bf16_burst"],
+        "peak_kind": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
+        "frac_of_sustained_peak": attn_tflops / peaks["bf16_sustained"],
+        "sustained_peak_sm_mhz": peaks.get("sustained_sm_mhz"),
         "traffic": traffic,
         "algorithmic_flop_per_launch": flops,
     }
@@ -661,26 +667,42 @@ def main():
 
     out_ref = out.clone()  # the p-run's O, before the dense run reuses `out`
 
-    # dense p = 1 reference: the same kernel over an all-blocks CSR
+    # dense p = 1 reference: the same kernel over an all-blocks CSR.  The part
+    # runs at its power cap, so the sparse step and the dense run are timed
+    # alternately (three rounds, each about 0.5 s of back-to-back work per
+    # arm, the last round kept) so that both see the same clocks.
     if not args.no_dense:
         rp_all = (torch.arange(rows + 1, device=dev, dtype=torch.int64) * nB).to(torch.int32)
         col_all = torch.arange(nB, device=dev, dtype=torch.int32).repeat(rows)
         attend(rp_all, col_all)
         torch.cuda.synchronize(dev)
-        kd = max(2, args.steps // 3)
-        ed = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(kd)]
-        for e in ed:
-            e[0].record(stream); attend(rp_all, col_all); e[1].record(stream)
-        torch.cuda.synchronize(dev)
-        ms_dense = sum(e[0].elapsed_time(e[1]) for e in ed) / kd
+
+        def back_to_back(fn, reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            return a.elapsed_time(b) / reps
+
+        ms_step_mean = sum(t_step) / len(t_step)
+        k_sparse = max(3, int(500.0 / max(ms_step_mean, 1e-3)))
+        k_dense = 4
+        for _ in range(3):
+            ms_sparse_alt = back_to_back(lambda: (search(), attend(), finish()), k_sparse)
+            ms_dense = back_to_back(lambda: attend(rp_all, col_all), k_dense)
         red = dense_flops / flops
         line["speedup_vs_p1"] = {
             "dense_attn_ms": ms_dense,
             "dense_attn_tflops": dense_flops / (ms_dense * 1e-3) / 1e12,
+            "sparse_step_ms_alternated": ms_sparse_alt,
             "attn_only": ms_dense / ms_attn,
-            "pipeline": ms_dense / (sum(t_step) / len(t_step)),
+            "pipeline": ms_dense / ms_sparse_alt,
             "executed_flop_reduction": red,
-            "pipeline_over_reduction": ms_dense / (sum(t_step) / len(t_step)) / red,
+            "pipeline_over_reduction": ms_dense / ms_sparse_alt / red,
+            "timing": f"alternated: {k_sparse} sparse steps then {k_dense} dense runs, "
+                      "3 rounds, last kept",
         }
         del rp_all, col_all
 

@@ -23,7 +23,7 @@ LIB = os.path.join(PKG, "libdsa.so")
 
 SOURCES = ["dsa_api.cu", "pool_score.cu", "select_topp.cu", "attn_sm100.cu",
            "attn_simt.cu", "block_mass.cu", "select_static.cu", "reorder.cu",
-           "attn_bwd.cu", "attn_bwd_sm100.cu"]
+           "attn_bwd.cu", "attn_bwd_sm100.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -58,7 +58,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // barriers (8 bytes each)
 // (kBarS, kBarP: one per half of the block's columns)
-enum : int { kBarFixed = 0, kBarRing = 1, kBarFree = 3, kBarS = 5, kBarP = 7, kNumBars = 9 };
+// (kBarDrain: teardown after an abort, every MMA issued is done)
+enum : int { kBarFixed = 0, kBarRing = 1, kBarFree = 3, kBarS = 5, kBarP = 7, kBarDrain = 9,
+             kNumBars = 10 };
 
 template <int D>
 struct BwdSmem {
@@ -140,6 +142,28 @@ __device__ __forceinline__ void mma_grad_half(uint32_t d, uint32_t a, uint64_t b
   }
 }
 
+// After a role gave up, copies and MMAs may still be in flight: the MMA
+// issuer commits once more and waits (bounded) until every MMA it issued is
+// done, the loader waits for the fixed tiles and its last ring loads, then
+// the whole CTA meets before shared and tensor memory are released.  Called
+// by every thread of the CTA.
+template <typename Bar>
+__device__ __forceinline__ void drain_after_abort(int warp, int lane, int n, int issued, Bar bar) {
+  if (warp == kMmaWarp && n > 0) {
+    if (lane == 0) {
+      mma_commit(bar(kBarDrain));
+      mbar_wait(bar(kBarDrain), 0u);
+    }
+    __syncwarp();
+  } else if (warp == kLoadWarp && lane == 0 && n > 0) {
+    for (int b = issued - 2 > 0 ? issued - 2 : 0; b < issued; ++b)
+      mbar_wait(bar(kBarRing + (b & 1)), (uint32_t)(b >> 1) & 1u);
+    mbar_wait(bar(kBarFixed), 0u);
+  }
+  tc_fence_before();
+  __syncthreads();
+}
+
 // Stores 32 fp32 accumulator columns of this thread's row, times `mul`, as bf16.
 __device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const uint32_t (&g)[32], float mul) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -212,11 +236,11 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n = s1 - s0;
+  int issued = 0;  // loader: blocks whose ring loads were issued
 
   if (warp == kLoadWarp) {
     if (lane == 0 && n > 0) {
       bool ok = true;
-      int issued = 0;
       mbar_expect_tx(bar(kBarFixed), 2 * kTileBytes);
       tma_tile<D>(sQ, &tmQ, q0, bh, bar(kBarFixed));
       tma_tile<D>(sO, &tmO, q0, bh, bar(kBarFixed));
@@ -234,9 +258,6 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       if (!ok) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
-        for (int b = issued - 2 > 0 ? issued - 2 : 0; b < issued; ++b)
-          mbar_wait(bar(kBarRing + (b & 1)), (uint32_t)(b >> 1) & 1u);
-        mbar_wait(bar(kBarFixed), 0u);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -366,6 +387,7 @@ bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) drain_after_abort(warp, lane, n, issued, bar);
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -425,11 +447,11 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   const uint32_t tmem = *tmem_slot;
   const int t0 = t_row_ptr[r];
   const int n = t_row_ptr[r + 1] - t0;  // built by the mask transpose: ascending, in range
+  int issued = 0;  // loader: blocks whose ring loads were issued
 
   if (warp == kLoadWarp) {
     if (lane == 0 && n > 0) {
       bool ok = true;
-      int issued = 0;
       mbar_expect_tx(bar(kBarFixed), 2 * kTileBytes);
       tma_tile<D>(sK, &tmK, k0, bh, bar(kBarFixed));
       tma_tile<D>(sV, &tmV, k0, bh, bar(kBarFixed));
@@ -446,9 +468,6 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       if (!ok) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
-        for (int b = issued - 2 > 0 ? issued - 2 : 0; b < issued; ++b)
-          mbar_wait(bar(kBarRing + (b & 1)), (uint32_t)(b >> 1) & 1u);
-        mbar_wait(bar(kBarFixed), 0u);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -588,6 +607,7 @@ bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) drain_after_abort(warp, lane, n, issued, bar);
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

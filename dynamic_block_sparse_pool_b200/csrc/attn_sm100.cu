@@ -80,7 +80,8 @@ enum : int {
   kBarSFull = kBarVFull + kStages,      // + stage: S(it) done
   kBarPFull = kBarSFull + kStages,      // + stage: P(it) written (one arrival per softmax warp)
   kBarPVDone = kBarPFull + kStages,     // + stage: PV(it) done
-  kNumBars = kBarPVDone + kStages
+  kBarDrain = kBarPVDone + kStages,     // teardown after an abort: every MMA issued is done
+  kNumBars = kBarDrain + 1
 };
 
 template <int D>
@@ -193,6 +194,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     s1 = s0;
   }
   const int n = s1 - s0;
+  int k_issued = 0, v_issued = 0;  // loader: blocks whose K / V loads were issued
 
   if (warp == kLoadWarp) {
     // ---------------------------------------------------------------- loader
@@ -202,7 +204,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       // is done, so K gets about three block periods to arrive from L2.
       constexpr int kKLead = 2;
       bool ok = true;
-      int k_issued = 0, v_issued = 0;  // blocks whose K / V loads were issued
       mbar_expect_tx(bar(kBarQ), kTileBytes);
       tma_tile<D>(sQ, &tmQ, q0, bh, bar(kBarQ));
       for (int step = 0; step < n + kKLead && ok; ++step) {
@@ -230,12 +231,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (!ok) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
-        // let the loads still in flight land before shared memory is released
-        for (int b = k_issued - kStages > 0 ? k_issued - kStages : 0; b < k_issued; ++b)
-          mbar_wait(bar(kBarKFull + b % kStages), (uint32_t)(b / kStages) & 1u);
-        for (int b = v_issued - kStages > 0 ? v_issued - kStages : 0; b < v_issued; ++b)
-          mbar_wait(bar(kBarVFull + b % kStages), (uint32_t)(b / kStages) & 1u);
-        mbar_wait(bar(kBarQ), 0u);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -524,6 +519,25 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // A role gave up: copies and MMAs may still be in flight.  Let every one
+    // of them finish (bounded) before shared and tensor memory are released.
+    if (warp == kMmaWarp && n > 0) {
+      if (lane == 0) {
+        mma_commit(bar(kBarDrain));  // arrives once all MMAs issued so far are done
+        mbar_wait(bar(kBarDrain), 0u);
+      }
+      __syncwarp();
+    } else if (warp == kLoadWarp && lane == 0 && n > 0) {
+      for (int b = k_issued - kStages > 0 ? k_issued - kStages : 0; b < k_issued; ++b)
+        mbar_wait(bar(kBarKFull + b % kStages), (uint32_t)(b / kStages) & 1u);
+      for (int b = v_issued - kStages > 0 ? v_issued - kStages : 0; b < v_issued; ++b)
+        mbar_wait(bar(kBarVFull + b % kStages), (uint32_t)(b / kStages) & 1u);
+      mbar_wait(bar(kBarQ), 0u);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

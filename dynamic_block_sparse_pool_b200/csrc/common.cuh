@@ -82,6 +82,8 @@ cudaError_t launch_attn_bwd_sm100(const void* q, const void* k, const void* v, c
                                   float scale, const int32_t* row_ptr, const int32_t* col_idx,
                                   const int32_t* t_row_ptr, const int32_t* t_col, void* dq, void* dk,
                                   void* dv, unsigned* err, cudaStream_t s);
+// One CTA that waits on an mbarrier nobody arrives at, with the given limit.
+cudaError_t launch_wait_timeout(unsigned long long limit_ns, unsigned* err, cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

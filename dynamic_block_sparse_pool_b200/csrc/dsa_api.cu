@@ -378,6 +378,19 @@ dsa_status dsa_permute_tokens(const void* src, void* dst, dsa_dtype dt, int B, i
   return DSA_OK;
 }
 
+dsa_status dsa_selftest_wait_timeout(unsigned long long limit_ns, void* stream) {
+  g_last_error.clear();
+  if (limit_ns < 1000ull || limit_ns > dsa::kWaitLimitNs)
+    return fail(DSA_ERR_INVALID_ARG, "limit_ns must be in [1000, %llu] (got %llu)",
+                dsa::kWaitLimitNs, limit_ns);
+  DeviceInfo* dev = nullptr;
+  dsa_status st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  cudaError_t e = dsa::launch_wait_timeout(limit_ns, dev->err_word, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait_timeout launch");
+  return DSA_OK;
+}
+
 dsa_status dsa_device_status(void* stream) {
   g_last_error.clear();
   DeviceInfo* dev = nullptr;
@@ -392,11 +405,12 @@ dsa_status dsa_device_status(void* stream) {
   const unsigned zero = 0;
   e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
   if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
-  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s%s", word,
+  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s%s%s", word,
               (word & dsa::kErrCsrIndex) ? " csr-index-out-of-range" : "",
               (word & dsa::kErrRowPtr) ? " bad-row-ptr" : "",
               (word & dsa::kErrProb) ? " probability-outside-[0,1]" : "",
               (word & dsa::kErrTimeout) ? " wait-timeout" : "",
+              (word & dsa::kErrAlign) ? " shared-memory-misaligned" : "",
               (word & dsa::kErrPerm) ? " permutation-index-out-of-range" : "");
 }
 

@@ -253,6 +253,13 @@ class HilbertOrder:
         return permute_tokens(x, self.perm, True, out)
 
 
+def selftest_wait_timeout(limit_ns: int = 1_000_000, device: Optional[torch.device] = None) -> None:
+    """Launch the failure-detection self-test: a bounded wait that runs out
+    after limit_ns and records a wait timeout (dsa_device_status then raises)."""
+    s = torch.cuda.current_stream(device).cuda_stream
+    check(lib().dsa_selftest_wait_timeout(int(limit_ns), s), "dsa_selftest_wait_timeout")
+
+
 def device_status(device: Optional[torch.device] = None) -> None:
     """Synchronises the current stream and raises DSAError if a kernel flagged bad input."""
     s = torch.cuda.current_stream(device).cuda_stream

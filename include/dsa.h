@@ -327,6 +327,23 @@ dsa_status dsa_select_topp_static(const float* probs, int rows, int nB, float p,
                                   int32_t* row_ptr, int32_t* col_idx, void* stream);
 
 /*
+ * Failure-detection self-test.  (No counterpart in the papers: it checks
+ * that this library's kernels report a stall instead of hanging.)
+ * Launches one CTA on `stream` that waits, with a limit of `limit_ns`
+ * nanoseconds, on a shared-memory mbarrier that nothing ever arrives at --
+ * the same bounded wait every tensor-core kernel of the library uses -- so
+ * the wait runs out, the kernel records a wait timeout in the device error
+ * word and returns.  It copies nothing, issues no MMA and
+ * holds no tensor memory.  After it, dsa_device_status returns
+ * DSA_ERR_DEVICE with "wait-timeout" in dsa_last_error, and the device
+ * stays usable.
+ *
+ *   limit_ns   1000 .. 1e9 (the library's own limit for one wait).
+ * Errors: DSA_ERR_INVALID_ARG for a limit outside that range.
+ */
+dsa_status dsa_selftest_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the library's device-side
  * error word.  Returns DSA_OK, DSA_ERR_DEVICE (details in dsa_last_error)
  * or DSA_ERR_CUDA.

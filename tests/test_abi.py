@@ -52,6 +52,7 @@ def _ctype_of(c):
     if c.endswith("*"):
         return ctypes.c_char_p if c == "const char *" else ctypes.c_void_p
     return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+            "unsigned long long": ctypes.c_ulonglong,
             "dsa_dtype": ctypes.c_int, "dsa_status": ctypes.c_int}[c]
 
 
@@ -166,6 +167,12 @@ def test_pool_score_hier_rejects(lib):
     assert lib.dsa_pool_score_hier(*big) == _lib.DSA_ERR_INVALID_ARG
     assert lib.dsa_workspace_size(_lib.DSA_OP_POOL_SCORE_HIER2, 1, 2, 256, 64, 128) == \
         4 * (2 * 2 * 4 * 64 + 2 * 4 * 4)
+
+
+@pytest.mark.parametrize("limit", [0, 999, 10 ** 9 + 1, 2 ** 63])
+def test_selftest_wait_timeout_rejects_limits(lib, limit):
+    assert lib.dsa_selftest_wait_timeout(limit, None) == _lib.DSA_ERR_INVALID_ARG
+    assert "limit_ns" in lib.dsa_last_error().decode()
 
 
 def test_python_wrapper_fails_loudly_without_library(monkeypatch, tmp_path):

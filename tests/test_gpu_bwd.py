@@ -1,8 +1,11 @@
 """Backward of the block-sparse attention on the GPU against the fp64
 oracle's chain rule, for the pipeline's own masks, for random fixed masks
 (ragged tails, empty rows) and for a hand-built mask with an empty row and a
-key block nobody selects.  The oracle takes the row term from the same stored
-forward output O that the kernel receives.  bf16 with blocks of 128 runs on
+key block nobody selects.  The forward output O and lse that the kernel
+receives are the oracle's own (fp64, rounded to the input dtype and fp32), so
+no input of the comparison comes from the CUDA path; one test also runs the
+backward on the GPU forward's O and lse, as a caller would.  The oracle takes
+the row term from the same stored O that the kernel receives.  bf16 with blocks of 128 runs on
 the tensor-core kernels (P and dS as bf16 hi + lo terms), fp32 and blocks of
 64 on the fp32 CUDA-core kernels; both meet the same gates.
 
@@ -42,6 +45,24 @@ def _check_grads(q, k, v, dO, block, scale, rp, col, grads, out):
                 assert np.all(err <= np.abs(r) / 128 + 2e-3 * m), (name, bh, err.max(), m)
 
 
+def oracle_forward(q, k, v, block, scale, rp, col):
+    """The oracle's O (rounded to q's dtype) and lse (fp32) on the given mask,
+    as CUDA tensors: the stored forward outputs the backward receives."""
+    B, H, N, D = q.shape
+    nB = ops.n_blocks(N, block)
+    rp_c, col_c = rp.cpu().numpy().astype(np.int64), col.cpu().numpy().astype(np.int64)
+    out = torch.empty(q.shape, dtype=torch.float64)
+    lse = torch.empty(B, H, N, dtype=torch.float64)
+    for bh in range(B * H):
+        b, h = divmod(bh, H)
+        hrp, hcol, _ = head_csr(rp_c, col_c, bh, nB)
+        Oo, lo, _ = O.sparse_attention_head(np64(q[b, h]), np64(k[b, h]), np64(v[b, h]),
+                                            block, scale, hrp, hcol)
+        out[b, h] = torch.from_numpy(Oo)
+        lse[b, h] = torch.from_numpy(lo)
+    return out.to(q.dtype).cuda(), lse.float().cuda()
+
+
 @pytest.mark.parametrize("w", [synth.TINY, synth.SMALL], ids=lambda w: w.name)
 def test_backward_on_pipeline_mask(w):
     q, k, v = (t.cuda() for t in synth.make_qkv(w, 17))
@@ -49,11 +70,19 @@ def test_backward_on_pipeline_mask(w):
     sa = ops.sparse_attention(q, k, v, w.p[0], block=w.block, scale=scale)
     g = torch.Generator().manual_seed(3)
     dO = torch.randn(q.shape, generator=g).to(q.dtype).cuda()
+    nnz = int(sa.row_ptr[-1])
+    col = sa.col_idx[:nnz]
+    # the oracle's stored forward outputs on the pipeline's mask
+    out_o, lse_o = oracle_forward(q.cpu(), k.cpu(), v.cpu(), w.block, scale, sa.row_ptr, col)
+    grads = ops.attn_bwd(q, k, v, out_o, dO, lse_o, sa.row_ptr, sa.col_idx, w.block, scale)
+    ops.device_status()
+    _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), w.block, scale, sa.row_ptr, col, grads,
+                 out_o.cpu())
+    # and as a caller runs it: on the GPU forward's own O and lse
     grads = ops.attn_bwd(q, k, v, sa.out, dO, sa.lse, sa.row_ptr, sa.col_idx, w.block, scale)
     ops.device_status()
-    nnz = int(sa.row_ptr[-1])
-    _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), w.block, scale, sa.row_ptr,
-                 sa.col_idx[:nnz], grads, sa.out.cpu())
+    _check_grads(q.cpu(), k.cpu(), v.cpu(), dO.cpu(), w.block, scale, sa.row_ptr, col, grads,
+                 sa.out.cpu())
 
 
 @pytest.mark.parametrize("name,B,H,N,D,block,density", [
@@ -67,7 +96,7 @@ def test_backward_fixed_mask(name, B, H, N, D, block, density):
     nB = ops.n_blocks(N, block)
     rp, col = synth.random_csr(B * H * nB, nB, density, seed=5)
     scale = 1.0 / math.sqrt(D)
-    out, lse, _ = ops.attn_fwd(q, k, v, rp.cuda(), col.cuda(), block, scale)
+    out, lse = oracle_forward(q.cpu(), k.cpu(), v.cpu(), block, scale, rp, col)
     dO = torch.randn(q.shape, generator=torch.Generator().manual_seed(6)).to(q.dtype).cuda()
     grads = ops.attn_bwd(q, k, v, out, dO, lse, rp.cuda(), col.cuda(), block, scale)
     ops.device_status()
@@ -90,7 +119,7 @@ def test_backward_empty_row_unselected_block_and_repeatability():
     rp = torch.tensor(np.concatenate([[0], np.cumsum([len(r) for r in rows])]), dtype=torch.int32)
     col = torch.tensor(np.concatenate([np.array(r, dtype=np.int64) for r in rows]), dtype=torch.int32)
     rpg, colg = rp.cuda(), col.cuda()
-    out, lse, _ = ops.attn_fwd(q, k, v, rpg, colg, blk, scale)
+    out, lse = oracle_forward(q.cpu(), k.cpu(), v.cpu(), blk, scale, rp, col)
     dO = torch.randn(q.shape, generator=torch.Generator().manual_seed(8)).to(q.dtype).cuda()
     g1 = ops.attn_bwd(q, k, v, out, dO, lse, rpg, colg, blk, scale)
     g2 = ops.attn_bwd(q, k, v, out, dO, lse, rpg, colg, blk, scale)

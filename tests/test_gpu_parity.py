@@ -68,24 +68,27 @@ def check_select(P_gpu, p, rp_g, col_g, cand=None):
 
 def check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass, heads=None,
                     rows=None, tol=None):
-    """Oracle attention on the GPU's mask for the given heads / query-block rows."""
+    """Oracle attention on the GPU's mask for the given heads / query-block rows.
+
+    Only the sampled slices of the GPU outputs are copied to the host, so the
+    check stays cheap at full workload sizes (blk_lse alone is 7 GB at p = 1
+    on the Wan2.1-like grid)."""
     B, H, N, D = q.shape
     nB = ops.n_blocks(N, block)
     tol = tol or TOL[q.dtype]
     rp_c, col_c = rp.cpu().numpy().astype(np.int64), col.cpu().numpy().astype(np.int64)
-    out_c, lse_c = np64(out), lse.cpu().numpy().astype(np.float64)
-    blk_c, mass_c = blk.cpu().numpy().astype(np.float64), mass.cpu().numpy().astype(np.float64)
+    lse_c = lse.cpu().numpy().astype(np.float64)
     errs = []
     for bh in (range(B * H) if heads is None else heads):
         b, h = divmod(bh, H)
         hrp, hcol, base = head_csr(rp_c, col_c, bh, nB)
         Oo, lo, blo = O.sparse_attention_head(np64(q[b, h]), np64(k[b, h]), np64(v[b, h]),
                                               block, scale, hrp, hcol, rows=rows)
-        Mo = O.block_mass(lo, blo, hrp, N, block)
+        out_h = np64(out[b, h])
         sel_rows = range(nB) if rows is None else rows
         for i in sel_rows:
             a0, a1 = i * block, min(N, (i + 1) * block)
-            go, oo = out_c[b, h, a0:a1], Oo[a0:a1]
+            go, oo = out_h[a0:a1], Oo[a0:a1]
             errs.append(np.abs(go - oo).ravel())
             s0, s1 = int(hrp[i]), int(hrp[i + 1])
             if s1 == s0:
@@ -95,12 +98,18 @@ def check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass, heads=N
             np.testing.assert_allclose(lse_c[b, h, a0:a1], lo[a0:a1], rtol=0, atol=tol["lse"] * max(1.0, np.abs(lo[a0:a1]).max()),
                                        err_msg=f"lse head {bh} row {i}")
             # per-query block weights exp(blk_lse - lse) and the block masses
-            gq = np.exp(blk_c[base + s0:base + s1, :a1 - a0] - lse_c[b, h, a0:a1][None, :])
+            blk_g = np64(blk[base + s0:base + s1, :a1 - a0])
+            gq = np.exp(blk_g - lse_c[b, h, a0:a1][None, :])
             oq = np.exp(blo[s0:s1, :a1 - a0] - lo[a0:a1][None, :])
             np.testing.assert_allclose(gq, oq, rtol=0, atol=tol["qmass"], err_msg=f"blk_lse head {bh} row {i}")
-            np.testing.assert_allclose(mass_c[base + s0:base + s1], Mo[s0:s1], rtol=0, atol=tol["mass"],
+            # the oracle's mass of this one row (a CSR holding only row i)
+            rp_i = np.zeros(nB + 1, dtype=np.int64)
+            rp_i[i + 1:] = s1 - s0
+            Mo = O.block_mass(lo, blo[s0:s1], rp_i, N, block)
+            mass_g = np64(mass[base + s0:base + s1])
+            np.testing.assert_allclose(mass_g, Mo, rtol=0, atol=tol["mass"],
                                        err_msg=f"mass head {bh} row {i}")
-            np.testing.assert_allclose(mass_c[base + s0:base + s1].sum(), 1.0, atol=10 * tol["mass"])
+            np.testing.assert_allclose(mass_g.sum(), 1.0, atol=10 * tol["mass"])
     e = np.concatenate(errs) if errs else np.zeros(1)
     assert e.max() <= tol["o_max"], f"O max abs err {e.max():.3e}"
     assert e.mean() <= tol["o_mean"], f"O mean abs err {e.mean():.3e}"
@@ -266,10 +275,70 @@ def test_attention_fixed_mask(name, B, H, N, D, block, dtype, density, qscale):
     q = (q.float() * qscale).to(dtype)
     nB = ops.n_blocks(N, block)
     rows = B * H * nB
-    # empty rows in both slots of the row pairs the tensor-core kernel handles together
+    # empty rows, among them the first row of the grid
     empty = (0, 3) if rows > 4 else (1,) if rows > 2 else ()
     rp, col = _csr_with_empty(rows, nB, density, seed=4, empty=empty)
     scale, out, lse, blk, mass = run_fixed_mask(q, k, v, block, rp, col)
+    check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass)
+
+
+def _rereference_case():
+    """Q, K, V and a CSR whose rows list key blocks in an order that forces
+    the tensor-core kernel to change its softmax reference mid-row.
+
+    Keys are N(0, 0.3^2) plus b_j * (1, ..., 1) in key block j; queries are
+    N(0, 0.3^2) plus a_i * (1, ..., 1) in query block i.  With D = 128 and
+    scale 1/sqrt(128), block j then scores about 16.3 * a_i * b_j log2 units
+    above a cold block.  Rows where the kernel's first block is cold and a
+    later one is hot by >= 57 log2 units have partial sums >= 2^64 and must
+    redo that block against a new reference and rescale O; at >= 128 units
+    the unrescaled exponentials overflow fp32, so a missing redo would give
+    inf/NaN outputs instead of passing.  Head 1 negates the queries, so hot
+    blocks become very cold ones (blocks that underflow to zero).  Query rows
+    whose index is 3 mod 4, and rows 80-95 (one softmax warp's rows), carry
+    no a_i: some threads and a whole warp keep their reference while others
+    move it."""
+    D, block = 128, 128
+    N = 6 * block + 40                       # 7 blocks, the last one ragged (40 tokens)
+    nB = ops.n_blocks(N, block)
+    g = torch.Generator().manual_seed(77)
+    b_key = [0.0, 0.0, 1.0, 0.0, 0.0, 2.0, 3.0]
+    a_qry = [3.0, 4.0, 2.5, 6.0, 1.0, 5.0, 0.7]
+    k = 0.3 * torch.randn(N, D, generator=g)
+    q = 0.3 * torch.randn(N, D, generator=g)
+    for j in range(nB):
+        k[j * block:(j + 1) * block] += b_key[j]
+    for i in range(nB):
+        a = torch.full((min(N, (i + 1) * block) - i * block, 1), a_qry[i])
+        a[3::4] = 0.0
+        a[80:96] = 0.0
+        q[i * block:i * block + a.shape[0]] += a
+    v = torch.randn(N, D, generator=g)
+    q = torch.stack([q, -q])[None].to(torch.bfloat16)
+    k = torch.stack([k, k])[None].to(torch.bfloat16)
+    v = torch.stack([v, v.flip(0)])[None].to(torch.bfloat16)
+    orders = [
+        [0, 1, 3, 4, 5, 2, 6],   # hot block 5 at position 4; block 6 later, +49 (no redo)
+        [0, 2, 1, 5, 3, 4, 6],   # three successive redos: positions 1, 3 and 6
+        [6, 0, 1, 2, 3, 4, 5],   # hot ragged block first: no redo (control)
+        [0, 1, 3, 4, 6],         # ragged block last, ~290 units above: overflow redo
+        [4, 6, 0, 1, 2, 3, 5],   # low levels throughout (control)
+        [1, 3, 0, 4, 2, 6, 5],   # redo at position 4, overflow redo at 5
+        [0, 1, 2, 3, 4, 5, 6],
+    ]
+    rows = orders + orders                   # both heads
+    rp = torch.tensor([0] + list(torch.cumsum(torch.tensor([len(r) for r in rows]), 0)),
+                      dtype=torch.int32)
+    col = torch.tensor([c for r in rows for c in r], dtype=torch.int32)
+    return q, k, v, block, rp, col
+
+
+def test_attention_rereference_redo_and_rescale():
+    # GSRS abstract: exact attention weights within the FlashAttention pass.
+    # The lazy reference must stay exact when a later block dominates.
+    q, k, v, block, rp, col = _rereference_case()
+    scale, out, lse, blk, mass = run_fixed_mask(q, k, v, block, rp, col)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
     check_attention(q, k, v, block, scale, rp, col, out, lse, blk, mass)
 
 
@@ -296,8 +365,11 @@ def test_attention_dense_matches_textbook_and_column_order():
 # ------------------------------------------------------------ full pipeline --
 
 def pipeline_parity(w, seed, p, bandwidth=None, cand=None, heads=None, rows=None,
-                    prob_heads=None):
-    q, k, v = synth.make_qkv(w, seed, bandwidth=bandwidth)
+                    prob_heads=None, qkv=None):
+    """The whole pipeline on the GPU against the oracle: P on ``prob_heads``,
+    the CSR over every row, attention, lse, block log-sums and masses on
+    ``heads`` x ``rows``.  ``qkv`` reuses an earlier draw of the same inputs."""
+    q, k, v = synth.make_qkv(w, seed, bandwidth=bandwidth) if qkv is None else qkv
     scale = 1.0 / math.sqrt(w.head_dim)
     qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
     cand_g = None if cand is None else (cand[0].cuda(), cand[1].cuda())

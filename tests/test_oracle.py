@@ -334,6 +334,40 @@ def test_recall_is_one_at_p1_and_pipeline_reduced_equals_full():
     np.testing.assert_array_equal(full["O"], red["O"])
 
 
+def test_recall_zero_query_is_selected_key_fraction():
+    # q = 0: the dense softmax is uniform over all N keys, so a row's recall
+    # is (keys in its selected blocks) / N, whatever the keys are
+    N, Bs, D = 200, 64, 4           # blocks of 64, 64, 64 and 8 tokens
+    _, k, _ = _qkv(N, D, 12, scale=2.0)
+    q = np.zeros((N, D))
+    rp = np.array([0, 2, 2, 3, 4])  # row 1 selects nothing
+    col = np.array([0, 3, 3, 1])
+    r = O.recall(q, k, Bs, 0.7, rp, col)
+    np.testing.assert_allclose(r, [72 / 200, 0.0, 8 / 200, 64 / 200], rtol=1e-14)
+
+
+def test_recall_block_constant_keys_closed_form():
+    # keys constant within each block (k_u = c_j): a query's dense weight on
+    # block j is |B_j| e^{z_j} / sum_j' |B_j'| e^{z_j'} with z_j = s q.c_j, so
+    # recall_i = mean_t of the selected blocks' share.  Ragged sizes and
+    # distinct per-block logits make a wrong block index or size fail.
+    N, Bs, D, s = 200, 64, 3, 0.8
+    b = O.block_bounds(N, Bs)
+    rng = np.random.default_rng(13)
+    c = rng.normal(size=(len(b), D))
+    k = np.concatenate([np.tile(c[j], (b1 - b0, 1)) for j, (b0, b1) in enumerate(b)])
+    q = rng.normal(size=(N, D))
+    rp = np.array([0, 1, 3, 4, 6])
+    col = np.array([3, 0, 2, 1, 1, 3])
+    sizes = np.array([b1 - b0 for b0, b1 in b], dtype=np.float64)
+    r = O.recall(q, k, Bs, s, rp, col)
+    for i, (a0, a1) in enumerate(b):
+        z = s * (q[a0:a1] @ c.T)                      # [queries, blocks]
+        wts = sizes[None, :] * np.exp(z)
+        share = wts[:, col[rp[i]:rp[i + 1]]].sum(1) / wts.sum(1)
+        np.testing.assert_allclose(r[i], share.mean(), rtol=1e-12)
+
+
 def test_executed_flops_counts_ragged_blocks():
     rp = np.array([0, 2, 3])
     col = np.array([0, 1, 1])          # N = 100, Bs = 64: blocks of 64 and 36
