@@ -114,6 +114,67 @@ __device__ __forceinline__ float exp2_mufu(float x) {
   return y;
 }
 
+// Number of the 16 eight-key chunks of each thread's S row pair whose
+// exponentials run on the FMA pipe (exp2_poly_x2) instead of the MUFU.  Per
+// block the softmax needs 128 x 128 exponentials, 1024 MUFU cycles per SM at
+// 16 per clock: as much as the block's MMAs at D = 128 and twice theirs at
+// D = 64.  Measured, the MUFU is not what bounds this kernel (moving a
+// quarter or half of the exponentials to the FMA pipe made it slower at
+// both D), so by default every exponential runs on the MUFU.
+#ifndef DSA_POLY_CHUNKS_D64
+#define DSA_POLY_CHUNKS_D64 0
+#endif
+#ifndef DSA_POLY_CHUNKS_D128
+#define DSA_POLY_CHUNKS_D128 0
+#endif
+// Warps 4-7 start their first block once S(1) is ready (half a block behind
+// warps 0-3), so the two softmax warps of each SM sub-partition are out of
+// phase.
+#ifndef DSA_SOFTMAX_LAG
+#define DSA_SOFTMAX_LAG 1
+#endif
+template <int D>
+constexpr int poly_chunks() { return D == 64 ? DSA_POLY_CHUNKS_D64 : DSA_POLY_CHUNKS_D128; }
+// chunk k of 16 takes the polynomial path: the kPoly chunks are spread evenly
+__host__ __device__ constexpr bool poly_chunk(int k, int kPoly) {
+  return (k + 1) * kPoly / 16 != k * kPoly / 16;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe.  Range reduction in the
+// manner of Cody and Waite for base 2: x = j + r with j = round(x), taken by
+// adding the shifter 1.5 * 2^23 (the sum keeps j in its low mantissa bits)
+// and r = x - j in [-0.5, 0.5]; 2^r by the degree-4 polynomial of least
+// maximum relative error on [-0.5, 0.5] (Remez exchange, error 2.6e-6, 2.7e-6
+// when evaluated in fp32); 2^j by adding j to the exponent field of 2^r.  x is
+// clamped to [-126, 127] first, so the exponent stays in range: results
+// below 2^-126 come out as about 2^-126 instead of 0, and anything that
+// would overflow comes out at or above 2^126.5.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99999928474426270f, c1 = 0.69312179088592529f,
+                  c2 = 0.24024743318367004f, c3 = 0.055917859077453613f,
+                  c4 = 0.0095701022073626518f;
+  float x0, x1;
+  unpack_f32x2(x2, x0, x1);
+  x0 = fminf(fmaxf(x0, -126.0f), 127.0f);
+  x1 = fminf(fmaxf(x1, -126.0f), 127.0f);
+  const uint64_t xc = pack_f32x2(x0, x1);
+  const uint64_t t = add_f32x2(xc, pack_f32x2(kShift, kShift));     // shifter + j
+  const uint64_t j = add_f32x2(t, pack_f32x2(-kShift, -kShift));    // j, exactly
+  const uint64_t r = fma_f32x2(j, pack_f32x2(-1.0f, -1.0f), xc);    // x - j, exactly
+  uint64_t p = fma_f32x2(pack_f32x2(c4, c4), r, pack_f32x2(c3, c3));
+  p = fma_f32x2(p, r, pack_f32x2(c2, c2));
+  p = fma_f32x2(p, r, pack_f32x2(c1, c1));
+  p = fma_f32x2(p, r, pack_f32x2(c0, c0));
+  float t0, t1, p0, p1;
+  unpack_f32x2(t, t0, t1);
+  unpack_f32x2(p, p0, p1);
+  // (shifter + j) << 23 leaves j << 23 (the shifter's bits shift out)
+  const uint32_t e0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t e1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  return pack_f32x2(__uint_as_float(e0), __uint_as_float(e1));
+}
+
 template <int D>
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row, int bh,
                                          uint32_t bar) {
@@ -135,6 +196,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, true);
   constexpr uint32_t kTileBytes = L::kTile;
   constexpr int kHalfD = D / 2;   // O columns owned by each half of a row
+  constexpr int kPoly = poly_chunks<D>();
 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
@@ -324,9 +386,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     // except through PV(it) -> S(it + 3).  (S(4) cannot complete before these
     // warps have produced P(1), so the wait below sees the first phase of
     // buffer 1.)
+#if DSA_SOFTMAX_LAG
     if ((warp >> 2) == 1 && n > 1) {
       if (!warp_all(mbar_wait(bar(kBarSFull + 1), 0u))) failed = true;
     }
+#endif
     for (int it = 0; it < n && !failed; ++it) {
       const int b = it % kSBufs;
       const uint32_t tS = tmem + lane_off + 128u * (uint32_t)b;
@@ -363,12 +427,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           float a0, a1, b0, b1;
-          unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1])), sc2, na2), a0, a1);
-          unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3])), sc2, nb2), b0, b1);
-          a0 = exp2_mufu(a0);
-          a1 = exp2_mufu(a1);
-          b0 = exp2_mufu(b0);
-          b1 = exp2_mufu(b1);
+          const uint64_t xa = fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1])), sc2, na2);
+          const uint64_t xb = fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3])), sc2, nb2);
+          if (poly_chunk(k, kPoly)) {
+            unpack_f32x2(exp2_poly_x2(xa), a0, a1);
+            unpack_f32x2(exp2_poly_x2(xb), b0, b1);
+          } else {
+            unpack_f32x2(xa, a0, a1);
+            unpack_f32x2(xb, b0, b1);
+            a0 = exp2_mufu(a0);
+            a1 = exp2_mufu(a1);
+            b0 = exp2_mufu(b0);
+            b1 = exp2_mufu(b1);
+          }
           rsa2[k & 1] = add_f32x2(rsa2[k & 1], pack_f32x2(a0, a1));
           rsb2[k & 1] = add_f32x2(rsb2[k & 1], pack_f32x2(b0, b1));
           const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1);
