@@ -133,6 +133,11 @@ __device__ __forceinline__ float exp2_mufu(float x) {
 #ifndef DSA_SOFTMAX_LAG
 #define DSA_SOFTMAX_LAG 1
 #endif
+// sleep between polls of the MMA issuer's and the loader's waits (ns)
+#ifndef DSA_IDLE_SLEEP_NS
+#define DSA_IDLE_SLEEP_NS 0
+#endif
+constexpr uint32_t kIdleSleepNs = DSA_IDLE_SLEEP_NS;
 template <int D>
 constexpr int poly_chunks() { return D == 64 ? DSA_POLY_CHUNKS_D64 : DSA_POLY_CHUNKS_D128; }
 // chunk k of 16 takes the polynomial path: the kPoly chunks are spread evenly
@@ -273,7 +278,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           const int it = step, s = it % kStages;
           const int j = col_idx[s0 + it];
           // K slot s is free once S(it - 3) is done
-          ok = mbar_wait(bar(kBarSFull + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
+          ok = mbar_wait_idle(bar(kBarSFull + s), ((uint32_t)(it / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
           if (!ok) break;
           mbar_expect_tx(bar(kBarKFull + s), kTileBytes);
           tma_tile<D>(sK + s * kTileBytes, &tmK, j * BN, bh, bar(kBarKFull + s));
@@ -283,7 +288,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           const int it = step - kKLead, s = it % kStages;
           const int j = col_idx[s0 + it];
           // V slot s is free once PV(it - 3) is done
-          ok = mbar_wait(bar(kBarPVDone + s), ((uint32_t)(it / kStages) & 1u) ^ 1u) && !*abort_flag;
+          ok = mbar_wait_idle(bar(kBarPVDone + s), ((uint32_t)(it / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
           if (!ok) break;
           mbar_expect_tx(bar(kBarVFull + s), kTileBytes);
           tma_tile<D>(sV + s * kTileBytes, &tmV, j * BN, bh, bar(kBarVFull + s));
@@ -318,7 +323,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       // in the async proxy and are ordered by the mbarrier alone.
       auto issue_s = [&](int it, auto stage) {
         constexpr int s = decltype(stage)::value;
-        if (!(ok = ok && warp_all(mbar_wait(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u))))
+        if (!(ok = ok && warp_all(mbar_wait_idle(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u, kIdleSleepNs))))
           return;
         if (leader) {
           const uint32_t d = tmem + 128u * s;
@@ -334,8 +339,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       auto block = [&](int it, auto stage) {
         constexpr int s = decltype(stage)::value;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (!(ok = ok && warp_all(mbar_wait(bar(kBarPFull + s), ph)) &&
-                   warp_all(mbar_wait(bar(kBarVFull + s), ph))))
+        if (!(ok = ok && warp_all(mbar_wait_idle(bar(kBarPFull + s), ph, kIdleSleepNs)) &&
+                   warp_all(mbar_wait_idle(bar(kBarVFull + s), ph, kIdleSleepNs))))
           return;
         tc_fence_after();
         if (leader) {

@@ -65,6 +65,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// mbar_wait for a warp that has nothing else to do while it waits (the MMA
+// issuer, the TMA loader): between polls it sleeps for about sleep_ns, so
+// its polling does not compete with the softmax warps of its SM
+// sub-partition for issue slots and the shared-memory pipe.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    if (sleep_ns) __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // ------------------------------------------------------------------- TMA ----
 
 // 3-D tiled tensor load (no multicast) into shared memory, completion counted
