@@ -192,7 +192,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, int N, int nB,
+                      const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmO, int N, int nB,
                       float scale_log2, const int32_t* __restrict__ row_ptr,
                       const int32_t* __restrict__ col_idx, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ lse, float* __restrict__ blk_lse, unsigned* err) {
@@ -202,6 +203,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   constexpr uint32_t kTileBytes = L::kTile;
   constexpr int kHalfD = D / 2;   // O columns owned by each half of a row
   constexpr int kPoly = poly_chunks<D>();
+  constexpr bool kTmaStoreO = D == 128;  // O leaves through shared memory and one TMA store
 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
@@ -239,6 +241,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
+    prefetch_tensormap(&tmO);
   }
   __syncthreads();
 
@@ -543,6 +546,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
     }
 
+    bool o_ok = false;  // this warp's rows of O are in shared memory
     if (failed) {
       *abort_flag = 1;
       flag_error(err, kErrTimeout);
@@ -557,8 +561,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       } else {
         tc_fence_after();
         const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
-        __nv_bfloat16* oa = out + ((size_t)bh * N + q0 + ra) * D + 2 * t0;
-        __nv_bfloat16* ob = out + ((size_t)bh * N + q0 + rb) * D + 2 * t0;
+        // D = 128: O / l as bf16 into the Q tile's shared memory (every MMA,
+        // and so every read of Q, is done), in the 128-byte-swizzled layout
+        // of the tensor map (16-byte chunk k of row r sits at chunk
+        // k ^ (r % 8)), for one TMA store below.  D = 64: straight to global
+        // memory (measured faster there).
+        uint8_t* sa = smem + L::kQ + ra * 128 + 4 * t0;
+        uint8_t* sb = smem + L::kQ + rb * 128 + 4 * t0;
+        __nv_bfloat16* ga = out + ((size_t)bh * N + q0 + ra) * D + 2 * t0;
+        __nv_bfloat16* gb = out + ((size_t)bh * N + q0 + rb) * D + 2 * t0;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t o[32];
@@ -570,10 +581,17 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                             __uint_as_float(o[4 * k + 1]) * inv_a);
             const __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[4 * k + 2]) * inv_b,
                                                             __uint_as_float(o[4 * k + 3]) * inv_b);
-            if (ra < qlen) *reinterpret_cast<__nv_bfloat162*>(oa + 64 * c + 8 * k) = ha;
-            if (rb < qlen) *reinterpret_cast<__nv_bfloat162*>(ob + 64 * c + 8 * k) = hb;
+            if (kTmaStoreO) {
+              *reinterpret_cast<__nv_bfloat162*>(sa + c * L::kSub + ((k ^ (ra & 7)) << 4)) = ha;
+              *reinterpret_cast<__nv_bfloat162*>(sb + c * L::kSub + ((k ^ (rb & 7)) << 4)) = hb;
+            } else {
+              if (ra < qlen) *reinterpret_cast<__nv_bfloat162*>(ga + 64 * c + 8 * k) = ha;
+              if (rb < qlen) *reinterpret_cast<__nv_bfloat162*>(gb + 64 * c + 8 * k) = hb;
+            }
           }
         }
+        if (kTmaStoreO) fence_proxy_async_smem();
+        o_ok = true;
         if (t0 == 0 && lse != nullptr) {
           if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
           if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
@@ -589,6 +607,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (t0 == 0 && lse != nullptr) {
         if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = -INFINITY;
         if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = -INFINITY;
+      }
+    }
+    if (kTmaStoreO && n > 0) {
+      // Every softmax warp arrives here, the ones that gave up too, so none
+      // waits alone; then one thread stores the O tile with TMA (rows past N
+      // fall outside the tensor and are not written) and waits until the
+      // copy has read shared memory.
+      const bool any_fail = named_bar_or(1, kSoftmaxThreads, !o_ok);
+      if (!any_fail && tid == 0) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, sQ + c * L::kSub, c * 64, q0, bh);
+        tma_store_commit();
+        tma_store_wait_read();
       }
     }
   }
@@ -653,7 +684,8 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int D) {
 }
 
 template <int D>
-cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, int BH,
+cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mo, int BH,
                      int N, float scale, const int32_t* row_ptr, const int32_t* col_idx,
                      void* out, float* lse, float* blk_lse, unsigned* err, cudaStream_t s) {
   const int nB = ceil_div(N, BN);
@@ -664,7 +696,7 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   if (e != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
   attn_fwd_sm100_kernel<D><<<rows, kThreads, smem, s>>>(
-      mq, mk, mv, N, nB, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out), lse,
+      mq, mk, mv, mo, N, nB, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out), lse,
       blk_lse, err);
   return cudaGetLastError();
 }
@@ -675,14 +707,14 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int B
                               int D, float scale, const int32_t* row_ptr,
                               const int32_t* col_idx, void* out, float* lse, float* blk_lse,
                               unsigned* err, cudaStream_t s, const char** why) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_tile_map(&mq, q, BH, N, D) || !make_tile_map(&mk, k, BH, N, D) ||
-      !make_tile_map(&mv, v, BH, N, D)) {
+      !make_tile_map(&mv, v, BH, N, D) || !make_tile_map(&mo, out, BH, N, D)) {
     if (why) *why = "cuTensorMapEncodeTiled failed or is unavailable";
     return cudaErrorInvalidValue;
   }
-  if (D == 64) return launch_d<64>(mq, mk, mv, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, err, s);
-  return launch_d<128>(mq, mk, mv, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, err, s);
+  if (D == 64) return launch_d<64>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, err, s);
+  return launch_d<128>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, err, s);
 }
 
 }  // namespace dsa
