@@ -34,6 +34,7 @@ SIGNATURES = {
     "dsa_mass_to_probs": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
     "dsa_pool_score_hier": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "dsa_hilbert_order": (_i, [_i, _i, _i, _i, _vp]),
+    "dsa_gilbert_order": (_i, [_i, _i, _i, _i, _vp]),
     "dsa_permute_tokens": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp]),
     "dsa_select_topp_static": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]),
     "dsa_selftest_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),

@@ -15,6 +15,12 @@
 #include "common.cuh"
 #include "dsa.h"
 
+namespace dsa {
+// Grid cells of a T x H x W grid in generalised Hilbert walk order, as
+// row-major indices (t*H + y)*W + x (reorder.cu).
+bool generalised_hilbert_cells(int T, int H, int W, std::vector<int32_t>& grid_order);
+}  // namespace dsa
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -354,6 +360,22 @@ dsa_status dsa_hilbert_order(int T, int H, int W, int n_prefix, int32_t* perm) {
   std::sort(keys.begin(), keys.end());
   for (int i = 0; i < n_prefix; ++i) perm[i] = i;
   for (size_t i = 0; i < keys.size(); ++i) perm[n_prefix + i] = keys[i].second;
+  return DSA_OK;
+}
+
+dsa_status dsa_gilbert_order(int T, int H, int W, int n_prefix, int32_t* perm) {
+  g_last_error.clear();
+  if (!perm) return fail(DSA_ERR_INVALID_ARG, "null perm");
+  if (T < 1 || H < 1 || W < 1 || n_prefix < 0)
+    return fail(DSA_ERR_INVALID_ARG, "need T, H, W >= 1 and n_prefix >= 0");
+  if (std::max(T, std::max(H, W)) > (1 << 20)) return fail(DSA_ERR_INVALID_ARG, "grid side above 2^20");
+  const long long cells = (long long)T * H * W;
+  if (cells + n_prefix > 0x7fffffffLL) return fail(DSA_ERR_INVALID_ARG, "too many tokens");
+  std::vector<int32_t> grid;
+  if (!dsa::generalised_hilbert_cells(T, H, W, grid) || (long long)grid.size() != cells)
+    return fail(DSA_ERR_INVALID_ARG, "no walk for a %d x %d x %d grid", T, H, W);
+  for (int i = 0; i < n_prefix; ++i) perm[i] = i;
+  for (size_t i = 0; i < grid.size(); ++i) perm[n_prefix + i] = n_prefix + grid[i];
   return DSA_OK;
 }
 

@@ -220,6 +220,15 @@ def hilbert_order(T: int, H: int, W: int, n_prefix: int = 0) -> torch.Tensor:
     return perm
 
 
+def gilbert_order(T: int, H: int, W: int, n_prefix: int = 0) -> torch.Tensor:
+    """Host int32 [n_prefix + T*H*W]: perm[i] = original index of the token at
+    position i along the generalised Hilbert curve of the T x H x W grid
+    (consecutive grid tokens are grid neighbours; text prefix first)."""
+    perm = torch.empty(n_prefix + T * H * W, dtype=torch.int32)
+    check(lib().dsa_gilbert_order(T, H, W, n_prefix, perm.data_ptr()), "dsa_gilbert_order")
+    return perm
+
+
 def permute_tokens(x: torch.Tensor, perm: torch.Tensor, inverse: bool = False,
                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Gather (dst[i] = src[perm[i]]) or scatter (dst[perm[i]] = src[i]) of the
@@ -238,10 +247,15 @@ def permute_tokens(x: torch.Tensor, perm: torch.Tensor, inverse: bool = False,
 
 
 class HilbertOrder:
-    """The Hilbert token order of one grid, kept on the device."""
+    """The Hilbert token order of one grid, kept on the device.  curve:
+    "hilbert" (the enclosing power-of-two cube's curve, restricted to the
+    grid) or "gilbert" (the curve generalised to the grid's own box)."""
 
-    def __init__(self, T: int, H: int, W: int, n_prefix: int = 0, device=None):
-        self.host = hilbert_order(T, H, W, n_prefix)
+    def __init__(self, T: int, H: int, W: int, n_prefix: int = 0, device=None,
+                 curve: str = "hilbert"):
+        if curve not in ("hilbert", "gilbert"):
+            raise ValueError(f"unknown curve {curve!r}")
+        self.host = (hilbert_order if curve == "hilbert" else gilbert_order)(T, H, W, n_prefix)
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
         self.perm = self.host.to(dev)

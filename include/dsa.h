@@ -277,6 +277,29 @@ dsa_status dsa_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx, con
 dsa_status dsa_hilbert_order(int T, int H, int W, int n_prefix, int32_t* perm);
 
 /*
+ * Token order along a generalised Hilbert curve of the T x H x W grid itself
+ * (GSRS Figure 6: blocks along a Gilbert curve, the Hilbert curve extended
+ * to boxes of any size).  Host function, no device work.  Same perm
+ * convention and prefix rule as dsa_hilbert_order, but every two
+ * consecutive grid tokens are grid neighbours (one step in t, y or x), also
+ * on grids that are not power-of-two cubes.
+ *
+ * Construction (the pages give none): Hilbert's recursion on the box.  A
+ * walk of an a x b x c box runs from a corner to the corner a - 1 cells
+ * away along its first edge; it exists iff the box is one cell or a >= 2
+ * and not (a odd and b*c even).  The longest edge is split near its middle
+ * -- two boxes in a row along the travel edge, or a U-turn along another
+ * edge (two one-cell slabs when the travel edge is 2 long) -- at the first
+ * point, nearest the middle, whose parts all have walks.  The whole grid
+ * is walked from (0, 0, 0) along its longest edge that admits a walk.
+ *
+ *   perm       host, int32 [n_prefix + T*H*W].
+ * Errors: DSA_ERR_INVALID_ARG for null perm, non-positive sizes, a side
+ * above 2^20 or more than 2^31 - 1 tokens.
+ */
+dsa_status dsa_gilbert_order(int T, int H, int W, int n_prefix, int32_t* perm);
+
+/*
  * Reorders whole token rows of a [B, H, N, D] tensor by a permutation of N:
  *   inverse = 0 (gather):  dst[b, h, i, :] = src[b, h, perm[i], :]
  *   inverse = 1 (scatter): dst[b, h, perm[i], :] = src[b, h, i, :]

@@ -359,6 +359,103 @@ def hilbert_order(T: int, H: int, W: int, n_prefix: int = 0) -> np.ndarray:
     return np.array(list(range(n_prefix)) + [idx for _, idx in keys], dtype=np.int64)
 
 
+def _walk_feasible(a: int, b: int, c: int) -> bool:
+    """Whether an a x b x c box has a walk through every cell with unit
+    steps from one corner to the corner a - 1 cells away along the first
+    axis.  Colour the cells by the parity of their coordinate sum: a walk
+    alternates colours, so its two ends differ in colour iff it has an even
+    number of cells; the two corners differ in colour iff a is even.  Hence
+    a odd needs b * c odd.  A box of more than one cell also needs a >= 2
+    (the two ends must differ)."""
+    if a * b * c == 1:
+        return True
+    return a >= 2 and not (a % 2 == 1 and (b * c) % 2 == 0)
+
+
+def _nearest_first(n: int, lo: int, hi: int) -> List[int]:
+    """The integers of [lo, hi], closest to n first (the smaller first on a tie)."""
+    out = []
+    for d in range(0, hi - lo + 2):
+        for x in (n - d, n + d):
+            if lo <= x <= hi and x not in out:
+                out.append(x)
+    return out
+
+
+def _gilbert_walk(entry, U, V, W, out: list) -> None:
+    """Cells of one box in walk order, appended to out.
+
+    entry: the first cell (t, y, x).  U, V, W: the box's three edges as
+    (axis, direction +-1, length); the walk ends at entry + (len U - 1)
+    steps along U.  Hilbert's recursion generalised to any box: split the
+    longest edge near its middle, either
+      - along U into two boxes walked one after the other along U, or
+      - as a U-turn along an edge X (V or W): the part u < h, x < m walked
+        along +X, the part x >= m walked along U, and the part u >= h,
+        x < m walked back along -X (with two one-cell slabs when |U| = 2),
+    taking the first split point (nearest the middle) whose three or two
+    parts all admit their walks (_walk_feasible).  Consecutive cells are
+    always unit steps apart."""
+    a, b, c = U[2], V[2], W[2]
+
+    def at(p, edge, d):
+        q = list(p)
+        q[edge[0]] += edge[1] * d
+        return tuple(q)
+
+    if b == 1 and c == 1:
+        out.extend(at(entry, U, i) for i in range(a))
+        return
+    lens = {"U": a, "V": b, "W": c}
+    for name in sorted(lens, key=lambda k: (-lens[k], "UVW".index(k))):
+        if name == "U":
+            for a1 in _nearest_first(a // 2, 1, a - 1):
+                if _walk_feasible(a1, b, c) and _walk_feasible(a - a1, b, c):
+                    _gilbert_walk(entry, (U[0], U[1], a1), V, W, out)
+                    _gilbert_walk(at(entry, U, a1), (U[0], U[1], a - a1), V, W, out)
+                    return
+            continue
+        X, Y = (V, W) if name == "V" else (W, V)
+        x = X[2]
+        if a < 2 or x < 2:
+            continue
+        if a == 2 and _walk_feasible(x, 1, Y[2]):
+            _gilbert_walk(entry, X, (U[0], U[1], 1), Y, out)
+            _gilbert_walk(at(at(entry, U, 1), X, x - 1), (X[0], -X[1], x), (U[0], U[1], 1), Y, out)
+            return
+        for m in _nearest_first(x // 2, 1, x - 1):
+            for h in _nearest_first(a // 2, 1, a - 1):
+                if (_walk_feasible(m, h, Y[2]) and _walk_feasible(a, x - m, Y[2])
+                        and _walk_feasible(m, a - h, Y[2])):
+                    _gilbert_walk(entry, (X[0], X[1], m), (U[0], U[1], h), Y, out)
+                    _gilbert_walk(at(entry, X, m), U, (X[0], X[1], x - m), Y, out)
+                    _gilbert_walk(at(at(entry, U, a - 1), X, m - 1), (X[0], -X[1], m),
+                                  (U[0], -U[1], a - h), Y, out)
+                    return
+    raise ValueError(f"no walk for a {a} x {b} x {c} box")
+
+
+def gilbert_order(T: int, H: int, W: int, n_prefix: int = 0) -> np.ndarray:
+    """perm [n_prefix + T*H*W] along a generalised Hilbert curve of the
+    T x H x W grid itself (GSRS Figure 6: blocks along a Gilbert curve, a
+    Hilbert curve generalised to boxes of any size; the pages give no
+    construction, so this is the plain recursive one of _gilbert_walk).
+    Unlike hilbert_order, consecutive tokens are always grid neighbours.
+    The walk starts at cell (0, 0, 0) and travels along the longest axis
+    that admits a corner-to-corner walk (ties: t before y before x); the
+    text prefix keeps its leading positions."""
+    dims = (T, H, W)
+    for axis in sorted(range(3), key=lambda i: (-dims[i], i)):
+        rest = [j for j in range(3) if j != axis]
+        if _walk_feasible(dims[axis], dims[rest[0]], dims[rest[1]]):
+            break
+    cells: list = []
+    _gilbert_walk((0, 0, 0), (axis, 1, dims[axis]), (rest[0], 1, dims[rest[0]]),
+                  (rest[1], 1, dims[rest[1]]), cells)
+    grid = [n_prefix + (t * H + y) * W + x for t, y, x in cells]
+    return np.array(list(range(n_prefix)) + grid, dtype=np.int64)
+
+
 def dense_attention(q, k, v, scale: float):
     """Textbook softmax(scale * Q K^T) V over all N keys, fp64; also lse."""
     q = np.asarray(q, np.float64)

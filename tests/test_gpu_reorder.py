@@ -1,5 +1,6 @@
 """Token reordering on the GPU: the permutation kernel bit-exact, and the
-whole pipeline on Hilbert-ordered tokens against the oracle on the same
+whole pipeline on tokens ordered along the Hilbert curve (of the enclosing
+cube, or generalised to the grid's own box) against the oracle on the same
 reordered inputs (gates of test_gpu_parity)."""
 import math
 
@@ -36,10 +37,11 @@ def test_permute_tokens_flags_bad_entry():
         ops.device_status()
 
 
+@pytest.mark.parametrize("curve", ["hilbert", "gilbert"])
 @pytest.mark.parametrize("w", [synth.SMALL, synth.TINY], ids=lambda w: w.name)
-def test_pipeline_on_hilbert_order(w):
+def test_pipeline_on_hilbert_order(w, curve):
     q, k, v = synth.make_qkv(w, 7)
-    order = HilbertOrder(w.T, w.Hg, w.W, w.n_prefix)
+    order = HilbertOrder(w.T, w.Hg, w.W, w.n_prefix, curve=curve)
     perm = order.host.long()
     qg, kg, vg = (order.gather(t.cuda()) for t in (q, k, v))
     ops.device_status()

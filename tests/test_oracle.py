@@ -417,6 +417,81 @@ def test_hilbert_blocks_are_more_compact_than_row_major():
     assert extent(perm) < 0.5 * extent(np.arange(T * H * W))
 
 
+def _hamiltonian_corner_walk_exists(a, b, c):
+    """Brute force: is there a path through every cell of an a x b x c box
+    (axes t, y, x) with unit steps from (0, 0, 0) to (a - 1, 0, 0)?"""
+    n = a * b * c
+    start, goal = (0, 0, 0), (a - 1, 0, 0)
+    seen = {start}
+
+    def dfs(p):
+        if len(seen) == n:
+            return p == goal
+        for d in ((1, 0, 0), (-1, 0, 0), (0, 1, 0), (0, -1, 0), (0, 0, 1), (0, 0, -1)):
+            q = (p[0] + d[0], p[1] + d[1], p[2] + d[2])
+            if 0 <= q[0] < a and 0 <= q[1] < b and 0 <= q[2] < c and q not in seen:
+                if q == goal and len(seen) + 1 < n:
+                    continue
+                seen.add(q)
+                if dfs(q):
+                    return True
+                seen.discard(q)
+        return False
+
+    return dfs(start)
+
+
+def test_gilbert_walk_feasibility_rule_is_exact_on_small_boxes():
+    # the two-colouring rule used to choose splits, against exhaustive search
+    for a, b, c in itertools.product(range(1, 4), range(1, 4), range(1, 3)):
+        if a * b * c > 12:
+            continue
+        assert O._walk_feasible(a, b, c) == _hamiltonian_corner_walk_exists(a, b, c), (a, b, c)
+
+
+def _gilbert_cells(T, H, W, P=0):
+    perm = O.gilbert_order(T, H, W, P)
+    assert perm[:P].tolist() == list(range(P))
+    assert sorted(perm.tolist()) == list(range(P + T * H * W))
+    return _cells(perm, H, W, P)
+
+
+def test_gilbert_is_a_unit_step_walk_on_every_small_box():
+    # GSRS Figure 6: a Hilbert curve generalised to boxes of any size; every
+    # box up to 7 x 7 x 7, including odd and one-cell-thick ones
+    for T, H, W in itertools.product(range(1, 8), repeat=3):
+        c = _gilbert_cells(T, H, W, 2)
+        if len(c) > 1:
+            assert np.all(np.abs(np.diff(c, axis=0)).sum(1) == 1), (T, H, W)
+        assert tuple(c[0]) == (0, 0, 0)
+        # it ends at the far corner along the longest walkable axis
+        dims = (T, H, W)
+        end = c[-1].tolist()
+        assert sum(1 for d, e in zip(dims, end) if e != 0) <= 1
+        moved = [i for i in range(3) if end[i] != 0]
+        if moved:
+            assert end[moved[0]] == dims[moved[0]] - 1
+
+
+@pytest.mark.parametrize("T,H,W,P", [(21, 45, 80, 0), (33, 45, 80, 0), (13, 30, 45, 226),
+                                     (8, 16, 16, 0), (4, 8, 8, 0)])
+def test_gilbert_workload_grids_walk_and_are_compact(T, H, W, P):
+    c = _gilbert_cells(T, H, W, P)
+    assert np.all(np.abs(np.diff(c, axis=0)).sum(1) == 1)
+    def spread(cells, Bs=128):
+        out = []
+        for a in range(0, len(cells), Bs):
+            blk = cells[a:a + Bs].astype(np.float64)
+            out.append(((blk - blk.mean(0)) ** 2).sum(1).mean())
+        return float(np.mean(out))
+    row_major = _cells(np.arange(P + T * H * W), H, W, P)
+    cube = _cells(O.hilbert_order(T, H, W, P), H, W, P)
+    # about as compact as the enclosing cube's curve, more than row-major
+    # (far more once a row of the grid is longer than a block)
+    assert spread(c) < 1.25 * spread(cube)
+    assert spread(c) < (0.1 if W * H > 128 * 8 else 0.9) * spread(row_major)
+
+
 # ----------------------------------------------------- hierarchical scores ----
 
 def test_hier_probs_sub1_is_block_probs_and_rows_sum_to_one():
