@@ -398,16 +398,19 @@ def sweep(args):
         masks[p] = point(w, q, k, v, p, dense=dms)[:2]
     # the same point with the two-level (sub-block) estimate
     point(w, q, k, v, 0.9, dense=dms, label=w.name + " two-level estimate (sub 2)", hier_sub=2)
-    # the same point on Hilbert-ordered tokens (dense attention is order-free),
-    # plus the cost of gathering Q, K, V and scattering O
-    order = ops.HilbertOrder(w.T, w.Hg, w.W, w.n_prefix, device=dev)
-    qh, kh, vh = (order.gather(t) for t in (q, k, v))
-    oh = torch.empty_like(q)
-    perm_ms = timed(lambda: (order.gather(q, out=qh), order.gather(k, out=kh),
-                             order.gather(v, out=vh), order.scatter(qh, out=oh)), 3)
-    point(w, qh, kh, vh, 0.9, dense=dms, label=w.name + " hilbert order",
-          extra={"reorder_ms": perm_ms, "reorder_bytes": 8 * q.numel() * q.element_size()})
-    del qh, kh, vh, oh
+    # the same point on tokens in curve order (dense attention is
+    # order-free), plus the cost of gathering Q, K, V and scattering O: the
+    # enclosing cube's Hilbert curve, then the generalised curve of the grid
+    for curve in ("hilbert", "gilbert"):
+        order = ops.HilbertOrder(w.T, w.Hg, w.W, w.n_prefix, device=dev, curve=curve)
+        qh, kh, vh = (order.gather(t) for t in (q, k, v))
+        oh = torch.empty_like(q)
+        perm_ms = timed(lambda: (order.gather(q, out=qh), order.gather(k, out=kh),
+                                 order.gather(v, out=vh), order.scatter(qh, out=oh)), 3)
+        point(w, qh, kh, vh, 0.9, dense=dms, label=w.name + " " + curve + " order",
+              extra={"reorder_ms": perm_ms,
+                     "reorder_bytes": 8 * q.numel() * q.element_size()})
+        del qh, kh, vh, oh
     q1, k1, v1 = synth.make_qkv(w, 1, device="cuda")
     dms1 = dense_of(w, q1, k1, v1)
     point(w, q1, k1, v1, 0.7, dense=dms1, label=w.name + " seed1 full search")

@@ -16,8 +16,10 @@
  *   dsa_attn_bwd     gradients of the attention for a fixed mask.
  *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
  *                    exact attention weights (the next mask of a schedule).
- *   dsa_hilbert_order, dsa_permute_tokens  token reordering along a 3-D
- *                    Hilbert curve before the pipeline, and back after it.
+ *   dsa_hilbert_order, dsa_gilbert_order, dsa_permute_tokens  token
+ *                    reordering along a 3-D Hilbert curve (the enclosing
+ *                    cube's, or one generalised to the grid's own box) before
+ *                    the pipeline, and back after it.
  *
  * Sources: "Sparse Attention for Video Generation Acceleration via Growing
  * Sparsity and Reduced Search" (GSRS, arXiv 2610.21129): abstract (Top-p

@@ -443,8 +443,8 @@ def _hamiltonian_corner_walk_exists(a, b, c):
 
 def test_gilbert_walk_feasibility_rule_is_exact_on_small_boxes():
     # the two-colouring rule used to choose splits, against exhaustive search
-    for a, b, c in itertools.product(range(1, 4), range(1, 4), range(1, 3)):
-        if a * b * c > 12:
+    for a, b, c in itertools.product(range(1, 6), range(1, 5), range(1, 5)):
+        if a * b * c > 24:
             continue
         assert O._walk_feasible(a, b, c) == _hamiltonian_corner_walk_exists(a, b, c), (a, b, c)
 
