@@ -1,13 +1,18 @@
 // Block-sparse attention forward on Blackwell tensor cores (sm_100a):
 // TMA loads of the indexed K/V blocks, tcgen05 MMAs with fp32 accumulators
-// in tensor memory, online softmax on CUDA cores, warp-specialised.
+// in tensor memory, online softmax on CUDA cores, warp-specialised and
+// persistent.
 //
 // GSRS (arXiv 2610.21129), abstract: exact attention over the selected
 // blocks inside a FlashAttention-style pass that also yields the exact
 // per-block attention weights.  DSV (arXiv 2502.07590), abstract: the work
-// per query block is skewed, so every query block is its own work item.
+// per query block is skewed, so every query block is its own work item and
+// the work items are handed out dynamically.
 //
-// One CTA per CSR row (one query block of 128 rows).  320 threads:
+// One CTA per SM.  Each CTA takes CSR rows (one query block of 128 rows
+// each) from a ticket counter shared by the launch until none are left, so
+// a CTA that drew short rows takes more of them (the balance of one CTA per
+// row, without a CTA's start-up and tear-down cost per row).  384 threads:
 //   warps 0-7  softmax: warp w owns the 16 query rows (TMEM lanes)
 //              32*(w%4) + 16*(w/4) .. +15; thread t of it owns two rows
 //              (t/4 and t/4 + 8 of those) and, in every 8-key chunk, keys
@@ -15,18 +20,30 @@
 //              four threads of a quad share two rows and a row reduction is
 //              two quad shuffles; no warp waits for another
 //   warp  8    MMA issuer (one thread) and TMEM allocation (whole warp)
-//   warp  9    TMA loader (one thread)
-// Tensor memory (512 columns): three S buffers at columns 0, 128, 256 (S of
-// block it in buffer it % 3; P, packed bf16 pairs, overwrites the first 64
-// columns of its buffer) and O at column 384.
-// Shared memory: Q, a 3-deep K ring and a 3-deep V ring of [128 x D] tiles.
+//   warp  9    TMA loader of Q and K (one thread)
+//   warp 10    TMA loader of V and TMA store of O (one thread): the softmax
+//              warps leave a row's O in the V slot of the row's last block,
+//              which no MMA reads once that block's PV is done, and this
+//              thread stores it before the slot takes its next V tile
+//   warp 11    row scheduler: draws the next row, checks its column indices
+//              and marks its ragged key block while the current row runs
+// Tensor memory (512 columns): three S buffers at columns 0, 128, 256 and O
+// at column 384.  Shared memory: Q, a 3-deep K ring and a 3-deep V ring of
+// [128 x D] tiles (a V slot doubles as the staging tile of a row's O), two
+// row-descriptor slots.
 //
-// Pipeline.  The MMA thread issues S(0), S(1), S(2), then for every block
-//   PV(it) [after P(it) is ready], S(it+3)
-// so two S tiles are computed ahead of the softmax, and the softmax warps
-// go from block to block without waiting for the tensor cores.  tcgen05 MMAs
-// from one thread execute in order: S(it+3) overwrites buffer it % 3 only
-// after PV(it) has read P(it) from it.
+// Blocks are numbered g = 0, 1, 2, ... across all the rows a CTA takes, in
+// order; block g uses K/V ring stage g % 3 and S buffer g % 3, so the rings
+// and the MMA pipeline run on across row boundaries: the next row's Q and
+// first K tiles load while the current row's last blocks are still in the
+// softmax.  Within a row the MMA thread issues S(0), S(1), S(2), then for
+// every block PV(it) [after P(it) is ready], S(it+3); the next row's S(0..2)
+// follow its last PV.  tcgen05 MMAs from one thread execute in order, so
+// S(g+3) overwrites buffer g % 3 only after PV(g) has read P(g) from it, and
+// a row's first PV (which overwrites O) runs only after every softmax warp
+// has read the previous row's O (each warp reads it before it writes its
+// first P of the next row).  Q of a row loads once every S of the previous
+// rows is done.
 //
 // Online softmax with a lazy reference: the first block's row maxima set the
 // reference m_ref; later blocks form P = 2^(S*scale*log2e - m_ref) without
@@ -44,7 +61,8 @@
 // K/V tile of block j: one 3-D TMA box {64 cols, 128 rows, 1 head} per 64
 // columns of D over the tensor {D, N, B*H}: rows past N are zero-filled and
 // masked to -inf.  No multicast.  Every mbarrier wait is bounded; a timeout
-// sets the device error word and the CTA winds down.
+// sets the device error word and the CTA winds down (rows it drew and did
+// not finish are left unwritten; the error word reports it).
 #include <type_traits>
 
 #include "sm100.cuh"
@@ -54,34 +72,50 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;         // query rows per CTA (one query block)
+constexpr int BM = 128;         // query rows per block row
 constexpr int BN = 128;         // keys per key block
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
-constexpr int kMmaWarp = 8, kLoadWarp = 9;
+constexpr int kMmaWarp = 8, kKLoadWarp = 9, kVLoadWarp = 10, kSchedWarp = 11;
 constexpr int kStages = 3;      // depth of the K ring and of the V ring
 constexpr int kSBufs = 3;       // S/P buffers in tensor memory
+constexpr int kRowSlots = 2;    // row descriptors in flight (current, next)
+// warps that read a row descriptor: 8 softmax, the MMA issuer, two loaders
+constexpr int kRowUsers = kSoftmaxThreads / 32 + 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 384;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kPMax = 0x1p64f;  // partial row sums at or above this redo the block
 
-// mbarrier slots, one per ring stage (block it uses stage it % 3 of the K
-// and V rings and S buffer it % 3, so one barrier per event serves both the
-// ring and the buffer).  Each tcgen05.commit and each fence costs the tensor
-// pipe a few dozen cycles, so a block signals only two events:
-//   SFull:  S(it) is done -- S is ready for the softmax and K slot is free
-//   PVDone: PV(it) is done -- V slot is free, O holds blocks 0..it
+// mbarrier slots.  Block g uses stage g % 3 of the K and V rings and S
+// buffer g % 3, so one barrier per event serves both the ring and the
+// buffer.  Each tcgen05.commit and each fence costs the tensor pipe a few
+// dozen cycles, so a block signals only two events:
+//   SFull:  S(g) is done -- S is ready for the softmax and K slot is free
+//   PVDone: PV(g) is done -- V slot is free, O holds the row through g
 static_assert(kStages == kSBufs, "ring stages and S buffers share barriers");
 enum : int {
   kBarQ = 0,
   kBarKFull = 1,                        // + stage: K tile landed
   kBarVFull = kBarKFull + kStages,      // + stage: V tile landed
-  kBarSFull = kBarVFull + kStages,      // + stage: S(it) done
-  kBarPFull = kBarSFull + kStages,      // + stage: P(it) written (one arrival per softmax warp)
-  kBarPVDone = kBarPFull + kStages,     // + stage: PV(it) done
-  kBarDrain = kBarPVDone + kStages,     // teardown after an abort: every MMA issued is done
+  kBarSFull = kBarVFull + kStages,      // + stage: S(g) done
+  kBarPFull = kBarSFull + kStages,      // + stage: P(g) written (one arrival per softmax warp)
+  kBarPVDone = kBarPFull + kStages,     // + stage: PV(g) done
+  kBarRowFull = kBarPVDone + kStages,   // + slot: row descriptor written
+  kBarRowFree = kBarRowFull + kRowSlots,  // + slot: every user is done with it
+  kBarOStaged = kBarRowFree + kRowSlots,  // + (row % 3): the row's O is in shared memory
+  kBarDrain = kBarOStaged + kStages,    // teardown after an abort: every MMA issued is done
   kNumBars = kBarDrain + 1
+};
+
+// A row handed to the CTA.  r < 0: no rows left.  n = 0 for an empty row
+// and for a malformed one (flagged in the error word; O = 0, lse = -inf).
+struct RowDesc {
+  int r;               // CSR row (b*H + h)*nB + i
+  int s0;              // its first list position
+  int n;               // its number of blocks
+  int pad;
+  uint32_t ragged[32]; // bit e: list position e (< 1024) holds the ragged last key block
 };
 
 template <int D>
@@ -92,8 +126,8 @@ struct SmemLayout {
   static constexpr int kK = kTile;                        // K ring
   static constexpr int kV = kK + kStages * kTile;         // V ring
   static constexpr int kBar = kV + kStages * kTile;
-  static constexpr int kRagged = kBar + 8 * kNumBars;     // uint32 [32]: list positions of the ragged block
-  static constexpr int kSlot = kRagged + 32 * 4;          // TMEM base, abort flag
+  static constexpr int kRow = kBar + 8 * kNumBars;        // RowDesc [kRowSlots]
+  static constexpr int kSlot = kRow + kRowSlots * (int)sizeof(RowDesc);  // TMEM base, abort flag
   static constexpr int kBytes = kSlot + 16;
 };
 
@@ -180,6 +214,35 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
   return pack_f32x2(__uint_as_float(e0), __uint_as_float(e1));
 }
 
+// 4 x 4 transpose of 32-bit words across the four threads of a quad (lanes
+// 4q .. 4q+3, t = lane % 4): afterwards x[u] holds what thread u held in
+// x[t].  Two butterfly steps: transpose the 2 x 2 blocks (partner t ^ 1),
+// then swap the off-diagonal blocks (partner t ^ 2).
+__device__ __forceinline__ void quad_transpose(uint32_t (&x)[4], int t) {
+  const bool odd = (t & 1) != 0, high = (t & 2) != 0;
+  uint32_t s0 = odd ? x[0] : x[1], s1 = odd ? x[2] : x[3];
+  s0 = __shfl_xor_sync(0xffffffffu, s0, 1);
+  s1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+  if (odd) {
+    x[0] = s0;
+    x[2] = s1;
+  } else {
+    x[1] = s0;
+    x[3] = s1;
+  }
+  s0 = high ? x[0] : x[2];
+  s1 = high ? x[1] : x[3];
+  s0 = __shfl_xor_sync(0xffffffffu, s0, 2);
+  s1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+  if (high) {
+    x[0] = s0;
+    x[1] = s1;
+  } else {
+    x[2] = s0;
+    x[3] = s1;
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row, int bh,
                                          uint32_t bar) {
@@ -193,43 +256,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
-                      const __grid_constant__ CUtensorMap tmO, int N, int nB,
+                      const __grid_constant__ CUtensorMap tmO, int N, int nB, int rows,
                       float scale_log2, const int32_t* __restrict__ row_ptr,
                       const int32_t* __restrict__ col_idx, __nv_bfloat16* __restrict__ out,
-                      float* __restrict__ lse, float* __restrict__ blk_lse, unsigned* err) {
+                      float* __restrict__ lse, float* __restrict__ blk_lse,
+                      unsigned* __restrict__ tickets, unsigned* err) {
   using L = SmemLayout<D>;
   constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, true);
   constexpr uint32_t kTileBytes = L::kTile;
-  constexpr int kHalfD = D / 2;   // O columns owned by each half of a row
   constexpr int kPoly = poly_chunks<D>();
-  constexpr bool kTmaStoreO = D == 128;  // O leaves through shared memory and one TMA store
 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
   if (base & 1023u) {  // the swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) flag_error(err, kErrAlign);
+    if (threadIdx.x == 0) {
+      flag_error(err, kErrAlign);
+      // this CTA draws no rows; it still counts as finished
+      if (atomicAdd(&tickets[1], 1u) == gridDim.x - 1) {
+        atomicExch(&tickets[0], 0u);
+        atomicExch(&tickets[1], 0u);
+      }
+    }
     return;
   }
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV;
   const uint32_t bars = base + L::kBar;
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
-  uint32_t* ragged_bits = reinterpret_cast<uint32_t*>(smem + L::kRagged);
+  RowDesc* rdesc = reinterpret_cast<RowDesc*>(smem + L::kRow);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlot + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r = blockIdx.x;
-  const int bh = r / nB, qi = r - bh * nB;
-  const int q0 = qi * BM;
-  const int qlen = min(BM, N - q0);
   const int kv_last = N - (nB - 1) * BN;  // keys in the last (possibly ragged) block
 
-  if (tid < 32) ragged_bits[tid] = 0u;
   if (warp == kMmaWarp) {
     if (lane == 0) {
-      for (int i = 0; i < kNumBars; ++i)
-        mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kStages) ? kSoftmaxThreads / 32 : 1);
+      for (int i = 0; i < kNumBars; ++i) {
+        uint32_t count = 1;
+        if (i >= kBarPFull && i < kBarPFull + kStages) count = kSoftmaxThreads / 32;
+        if (i >= kBarRowFree && i < kBarRowFree + kRowSlots) count = kRowUsers;
+        if (i >= kBarOStaged && i < kBarOStaged + kStages) count = kSoftmaxThreads / 32;
+        mbar_init(bar(i), count);
+      }
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -237,67 +306,175 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kLoadWarp && lane == 0) {
+  if (warp == kKLoadWarp && lane == 0) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
+  }
+  if (warp == kVLoadWarp && lane == 0) {
     prefetch_tensormap(&tmV);
     prefetch_tensormap(&tmO);
   }
-  __syncthreads();
-
-  // validate the row and mark where the ragged last key block sits in it
-  int s0 = row_ptr[r], s1 = row_ptr[r + 1];
-  bool bad = s0 < 0 || s1 < s0;
-  if (!bad)
-    for (int e = s0 + tid; e < s1; e += kThreads) {
-      const int j = col_idx[e];
-      bad |= (j < 0 || j >= nB);
-      if (j == nB - 1 && kv_last < BN && e - s0 < 1024)
-        atomicOr(&ragged_bits[(e - s0) >> 5], 1u << ((e - s0) & 31));
-    }
   tc_fence_before();
-  const bool any_bad = __syncthreads_or(bad);
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (any_bad) {
-    if (tid == 0) flag_error(err, kErrCsrIndex | kErrRowPtr);
-    s1 = s0;
-  }
-  const int n = s1 - s0;
-  int k_issued = 0, v_issued = 0;  // loader: blocks whose K / V loads were issued
 
-  if (warp == kLoadWarp) {
-    // ---------------------------------------------------------------- loader
-    if (lane == 0 && n > 0) {
-      // K runs kKLead blocks ahead of V: S(it) needs K(it) a block earlier
-      // than PV(it) needs V(it), and K(it + 3)'s slot frees as soon as S(it)
-      // is done, so K gets about three block periods to arrive from L2.
-      constexpr int kKLead = 2;
+  // Row descriptor k sits in slot k % 2; RowFull(slot) completes its phase
+  // (k / 2) % 2 when the scheduler has written it, RowFree(slot) when its
+  // kRowUsers readers are done with it.
+  auto row_wait = [&](int k) {
+    return mbar_wait_idle(bar(kBarRowFull + (k & 1)), (uint32_t)(k >> 1) & 1u, kIdleSleepNs);
+  };
+  // Blocks issued by the loaders (for the teardown after an abort).
+  uint32_t k_issued = 0, v_issued = 0, q_issued = 0;
+  bool had_rows = false;  // the MMA issuer issued at least one MMA
+
+  if (warp == kSchedWarp) {
+    // -------------------------------------------------------------- scheduler
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int slot = k & 1;
+      // slot is free once row k - 2's readers are done with it
+      // (a row lasts microseconds: poll every quarter microsecond)
+      if (k >= kRowSlots)
+        ok = warp_all(mbar_wait_idle(bar(kBarRowFree + slot), (uint32_t)((k - kRowSlots) >> 1) & 1u,
+                                     256u));
+      if (*abort_flag) ok = false;
+      int r = 0;
+      if (lane == 0) r = ok ? (int)atomicAdd(&tickets[0], 1u) : rows;
+      r = __shfl_sync(0xffffffffu, r, 0);
+      RowDesc* d = rdesc + slot;
+      if (r >= rows) {
+        if (lane == 0) {
+          d->r = -1;
+          mbar_arrive(bar(kBarRowFull + slot));
+        }
+        break;
+      }
+      int s0 = row_ptr[r], s1 = row_ptr[r + 1];
+      bool bad = s0 < 0 || s1 < s0;
+      if (!bad) {
+        for (int e0 = s0; e0 < s1; e0 += 32) {
+          const int e = e0 + lane;
+          const int j = e < s1 ? col_idx[e] : 0;
+          bad |= j < 0 || j >= nB;
+          const uint32_t rag = __ballot_sync(0xffffffffu, e < s1 && j == nB - 1 && kv_last < BN);
+          const int w = (e0 - s0) >> 5;
+          if (lane == 0 && w < 32) d->ragged[w] = rag;
+        }
+      }
+      bad = __any_sync(0xffffffffu, bad);
+      if (lane == 0) {
+        if (bad) flag_error(err, kErrCsrIndex | kErrRowPtr);
+        d->r = r;
+        d->s0 = bad ? 0 : s0;
+        d->n = bad ? 0 : s1 - s0;
+        mbar_arrive(bar(kBarRowFull + slot));  // release: the descriptor is visible to the readers
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) flag_error(err, kErrTimeout);
+    }
+  } else if (warp == kKLoadWarp) {
+    // ------------------------------------------------------------ Q/K loader
+    if (lane == 0) {
       bool ok = true;
-      mbar_expect_tx(bar(kBarQ), kTileBytes);
-      tma_tile<D>(sQ, &tmQ, q0, bh, bar(kBarQ));
-      for (int step = 0; step < n + kKLead && ok; ++step) {
-        if (step < n) {
-          const int it = step, s = it % kStages;
+      uint32_t g = 0;  // blocks of the rows before this one
+      for (int k = 0; ok; ++k) {
+        ok = row_wait(k) && !*abort_flag;
+        if (!ok) break;
+        const RowDesc* d = rdesc + (k & 1);
+        const int r = d->r, s0 = d->s0, n = d->n;
+        if (r < 0) break;
+        mbar_arrive(bar(kBarRowFree + (k & 1)));
+        if (n == 0) continue;
+        const int bh = r / nB, q0 = (r - bh * nB) * BM;
+        // Q's buffer is free once every S of the earlier rows is done
+        if (g > 0) {
+          ok = mbar_wait_idle(bar(kBarSFull + (g - 1) % kStages), ((g - 1) / kStages) & 1u, kIdleSleepNs) &&
+               !*abort_flag;
+          if (!ok) break;
+        }
+        mbar_expect_tx(bar(kBarQ), kTileBytes);
+        tma_tile<D>(sQ, &tmQ, q0, bh, bar(kBarQ));
+        ++q_issued;
+        for (int it = 0; it < n; ++it, ++g) {
+          const uint32_t s = g % kStages;
           const int j = col_idx[s0 + it];
-          // K slot s is free once S(it - 3) is done
-          ok = mbar_wait_idle(bar(kBarSFull + s), ((uint32_t)(it / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
+          // K slot s is free once S(g - 3) is done
+          ok = mbar_wait_idle(bar(kBarSFull + s), ((g / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
           if (!ok) break;
           mbar_expect_tx(bar(kBarKFull + s), kTileBytes);
           tma_tile<D>(sK + s * kTileBytes, &tmK, j * BN, bh, bar(kBarKFull + s));
-          k_issued = it + 1;
+          k_issued = g + 1;
         }
-        if (step >= kKLead) {
-          const int it = step - kKLead, s = it % kStages;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(err, kErrTimeout);
+      }
+    }
+  } else if (warp == kVLoadWarp) {
+    // -------------------------------------------------------------- V loader
+    // Also stores O: the softmax warps leave a row's O (bf16, in the tensor
+    // map's 128-byte-swizzled layout) in the V slot of the row's last block,
+    // which no MMA reads any more, and this thread stores it with TMA before
+    // it loads the next V tile into that slot (or at the end).
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t g = 0;      // blocks of the rows so far
+      uint32_t orows = 0;  // rows with blocks so far
+      // rows whose O waits in a V slot, oldest first: at most three (their
+      // last blocks are among the three blocks before the next V load)
+      struct Pending {
+        uint32_t last, idx;  // the row's last block; its number among rows with blocks
+        int bh, q0;
+      };
+      Pending p0{}, p1{}, p2{};
+      int np = 0;
+      auto store_o = [&]() -> bool {  // the oldest pending row
+        if (!mbar_wait(bar(kBarOStaged + p0.idx % kStages), (p0.idx / kStages) & 1u)) return false;
+        const uint32_t src = sV + (p0.last % kStages) * kTileBytes;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, src + c * L::kSub, c * 64, p0.q0, p0.bh);
+        tma_store_commit();
+        tma_store_wait_read();  // the slot may be refilled now
+        p0 = p1;
+        p1 = p2;
+        --np;
+        return true;
+      };
+      for (int k = 0; ok; ++k) {
+        ok = row_wait(k) && !*abort_flag;
+        if (!ok) break;
+        const RowDesc* d = rdesc + (k & 1);
+        const int r = d->r, s0 = d->s0, n = d->n;
+        if (r < 0) break;
+        mbar_arrive(bar(kBarRowFree + (k & 1)));
+        if (n == 0) continue;
+        const int bh = r / nB;
+        for (int it = 0; it < n; ++it, ++g) {
+          const uint32_t s = g % kStages;
           const int j = col_idx[s0 + it];
-          // V slot s is free once PV(it - 3) is done
-          ok = mbar_wait_idle(bar(kBarPVDone + s), ((uint32_t)(it / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
+          // slot s last held V(g - 3); if that was a row's last block, the
+          // row's O is staged there
+          if (np > 0 && p0.last + kStages == g && !(ok = store_o())) break;
+          // V slot s is free once PV(g - 3) is done
+          ok = mbar_wait_idle(bar(kBarPVDone + s), ((g / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
           if (!ok) break;
           mbar_expect_tx(bar(kBarVFull + s), kTileBytes);
           tma_tile<D>(sV + s * kTileBytes, &tmV, j * BN, bh, bar(kBarVFull + s));
-          v_issued = it + 1;
+          v_issued = g + 1;
         }
+        if (!ok) break;
+        const Pending pr{g - 1, orows++, bh, (r - bh * nB) * BM};
+        if (np == 0) p0 = pr;
+        else if (np == 1) p1 = pr;
+        else p2 = pr;
+        ++np;
       }
+      while (ok && np > 0) ok = store_o();
       if (!ok) {
         *abort_flag = 1;
         flag_error(err, kErrTimeout);
@@ -306,76 +483,97 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issuer
     // The whole warp runs the loop, so the waits, descriptors and addresses
-    // stay warp-uniform; lane 0 issues each MMA and commit.  The issuing warp
-    // shares its SM sub-partition with two busy softmax warps, so every
-    // instruction it saves shortens the tensor pipe's gaps.  The block loop
-    // is unrolled by the ring depth, which makes every stage index and
-    // descriptor offset a compile-time constant.
-    if (n > 0) {
-      const bool leader = lane == 0;
-      // three base descriptors; every other one differs only in its start
-      // address field (address >> 4, 14 bits, no carry below 256 KB)
-      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t dk0 = smem_desc_sw128(sK, 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(sV, L::kSub, 1024);
-      auto kdesc = [](int kk) -> uint64_t {  // K step kk of a K-major tile
-        return (uint64_t)(((kk >> 2) * L::kSub + (kk & 3) * 32) >> 4);
-      };
-      bool ok = warp_all(mbar_wait(bar(kBarQ), 0u));
-      // S(it) = Q K^T into buffer it % 3.  The TMA load and the MMA both act
-      // in the async proxy and are ordered by the mbarrier alone.
-      auto issue_s = [&](int it, auto stage) {
-        constexpr int s = decltype(stage)::value;
-        if (!(ok = ok && warp_all(mbar_wait_idle(bar(kBarKFull + s), (uint32_t)(it / kStages) & 1u, kIdleSleepNs))))
-          return;
-        if (leader) {
-          const uint32_t d = tmem + 128u * s;
-          const uint64_t k0 = dk0 + (uint64_t)((s * kTileBytes) >> 4);
-          mma_ss(d, dq0 + kdesc(0), k0 + kdesc(0), kIdescS, 0u);
+    // stay warp-uniform; lane 0 issues each MMA and commit.  Each ring stage
+    // has its own copy of the block step, so stage indices and descriptor
+    // offsets are compile-time constants; a switch on g % 3 picks the copy.
+    const bool leader = lane == 0;
+    // three base descriptors; every other one differs only in its start
+    // address field (address >> 4, 14 bits, no carry below 256 KB)
+    const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(sK, 16, 1024);
+    const uint64_t dv0 = smem_desc_sw128(sV, L::kSub, 1024);
+    auto kdesc = [](int kk) -> uint64_t {  // K step kk of a K-major tile
+      return (uint64_t)(((kk >> 2) * L::kSub + (kk & 3) * 32) >> 4);
+    };
+    bool ok = true;
+    // S(g) = Q K^T into buffer g % 3.  The TMA load and the MMA both act in
+    // the async proxy and are ordered by the mbarrier alone.
+    auto issue_s = [&](uint32_t gs, auto stage) {
+      constexpr int s = decltype(stage)::value;
+      if (!(ok = ok && warp_all(mbar_wait_idle(bar(kBarKFull + s), (gs / kStages) & 1u, kIdleSleepNs))))
+        return;
+      if (leader) {
+        const uint32_t d = tmem + 128u * s;
+        const uint64_t k0 = dk0 + (uint64_t)((s * kTileBytes) >> 4);
+        mma_ss(d, dq0 + kdesc(0), k0 + kdesc(0), kIdescS, 0u);
 #pragma unroll
-          for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, dq0 + kdesc(kk), k0 + kdesc(kk), kIdescS);
-          mma_commit(bar(kBarSFull + s));
-        }
-        __syncwarp();
-      };
-      // O += P(it) V(it), P from tensor memory; then S(it + 3) into the same buffer
-      auto block = [&](int it, auto stage) {
-        constexpr int s = decltype(stage)::value;
-        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (!(ok = ok && warp_all(mbar_wait_idle(bar(kBarPFull + s), ph, kIdleSleepNs)) &&
-                   warp_all(mbar_wait_idle(bar(kBarVFull + s), ph, kIdleSleepNs))))
-          return;
-        tc_fence_after();
-        if (leader) {
-          const uint32_t p = tmem + 128u * s;
-          const uint64_t v0 = dv0 + (uint64_t)((s * kTileBytes) >> 4);
-          if (it == 0)
-            mma_ts(tmem + kTmemO, p, v0, kIdescO, 0u);
-          else
-            mma_ts_acc(tmem + kTmemO, p, v0, kIdescO);
+        for (int kk = 1; kk < D / 16; ++kk) mma_ss_acc(d, dq0 + kdesc(kk), k0 + kdesc(kk), kIdescS);
+        mma_commit(bar(kBarSFull + s));
+      }
+      __syncwarp();
+    };
+    // O (+)= P(g) V(g), P from tensor memory (the row's first block
+    // overwrites O); then S(g + 3) into the same buffer if the row has it
+    auto block = [&](uint32_t gb, bool first, bool more, auto stage) {
+      constexpr int s = decltype(stage)::value;
+      const uint32_t ph = (gb / kStages) & 1u;
+      if (!(ok = ok && warp_all(mbar_wait_idle(bar(kBarPFull + s), ph, kIdleSleepNs)) &&
+                 warp_all(mbar_wait_idle(bar(kBarVFull + s), ph, kIdleSleepNs))))
+        return;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t p = tmem + 128u * s;
+        const uint64_t v0 = dv0 + (uint64_t)((s * kTileBytes) >> 4);
+        if (first)
+          mma_ts(tmem + kTmemO, p, v0, kIdescO, 0u);
+        else
+          mma_ts_acc(tmem + kTmemO, p, v0, kIdescO);
 #pragma unroll
-          for (int kk = 1; kk < BN / 16; ++kk)
-            mma_ts_acc(tmem + kTmemO, p + kk * 8, v0 + (uint64_t)((kk * 2048) >> 4), kIdescO);
-          mma_commit(bar(kBarPVDone + s));
+        for (int kk = 1; kk < BN / 16; ++kk)
+          mma_ts_acc(tmem + kTmemO, p + kk * 8, v0 + (uint64_t)((kk * 2048) >> 4), kIdescO);
+        mma_commit(bar(kBarPVDone + s));
+      }
+      __syncwarp();
+      if (more) issue_s(gb + kStages, stage);
+    };
+    using S0 = std::integral_constant<int, 0>;
+    using S1 = std::integral_constant<int, 1>;
+    using S2 = std::integral_constant<int, 2>;
+    uint32_t g = 0, qrows = 0;
+    for (int k = 0; ok; ++k) {
+      ok = warp_all(row_wait(k));
+      if (!ok) break;
+      const RowDesc* d = rdesc + (k & 1);
+      const int r = d->r, n = d->n;
+      if (r < 0) break;
+      __syncwarp();
+      if (leader) mbar_arrive(bar(kBarRowFree + (k & 1)));
+      if (n == 0) continue;
+      ok = warp_all(mbar_wait(bar(kBarQ), qrows & 1u));
+      ++qrows;
+      had_rows = true;
+      for (int it = 0; it < 3 && it < n && ok; ++it) {
+        const uint32_t gs = g + it;
+        switch (gs % kStages) {
+          case 0: issue_s(gs, S0{}); break;
+          case 1: issue_s(gs, S1{}); break;
+          default: issue_s(gs, S2{}); break;
         }
-        __syncwarp();
-        if (it + kStages < n) issue_s(it + kStages, stage);
-      };
-      using S0 = std::integral_constant<int, 0>;
-      using S1 = std::integral_constant<int, 1>;
-      using S2 = std::integral_constant<int, 2>;
-      issue_s(0, S0{});
-      if (n > 1) issue_s(1, S1{});
-      if (n > 2) issue_s(2, S2{});
-      for (int it = 0; it < n && ok; it += kStages) {
-        block(it, S0{});
-        if (it + 1 < n) block(it + 1, S1{});
-        if (it + 2 < n) block(it + 2, S2{});
       }
-      if (!ok && leader) {
-        *abort_flag = 1;
-        flag_error(err, kErrTimeout);
+      for (int it = 0; it < n && ok; ++it) {
+        const uint32_t gb = g + it;
+        const bool more = it + kStages < n;
+        switch (gb % kStages) {
+          case 0: block(gb, it == 0, more, S0{}); break;
+          case 1: block(gb, it == 0, more, S1{}); break;
+          default: block(gb, it == 0, more, S2{}); break;
+        }
       }
+      g += n;
+    }
+    if (!ok && leader) {
+      *abort_flag = 1;
+      flag_error(err, kErrTimeout);
     }
   } else {
     // ------------------------------------------------------------- softmax
@@ -383,132 +581,149 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int t0 = lane & 3;
     const int ra = rbase + (lane >> 2), rb = ra + 8;         // this thread's two rows
     const uint32_t lane_off = (uint32_t)rbase << 16;
-    float mref_a = -INFINITY, mref_b = -INFINITY;  // reference maxima (log2 units)
-    float l_a = 0.f, l_b = 0.f;                    // this thread's share of the row sums
     bool failed = false;
-    // Warps 4-7 start half a block behind warps 0-3 (they begin once S(1) is
-    // ready, one S MMA later than S(0)), so the two softmax warps of each SM
-    // sub-partition are out of phase: one is in its exp2 stretch (MUFU-bound)
-    // while the other loads, reduces and stores.  The lag is stable: S is
-    // triple-buffered and the leading warps never wait for the trailing ones
-    // except through PV(it) -> S(it + 3).  (S(4) cannot complete before these
-    // warps have produced P(1), so the wait below sees the first phase of
-    // buffer 1.)
-#if DSA_SOFTMAX_LAG
-    if ((warp >> 2) == 1 && n > 1) {
-      if (!warp_all(mbar_wait(bar(kBarSFull + 1), 0u))) failed = true;
-    }
-#endif
-    for (int it = 0; it < n && !failed; ++it) {
-      const int b = it % kSBufs;
-      const uint32_t tS = tmem + lane_off + 128u * (uint32_t)b;
-      if (!warp_all(mbar_wait(bar(kBarSFull + b), (uint32_t)(it / kSBufs) & 1u))) {
+    uint32_t g = 0;      // blocks of the rows so far
+    uint32_t orows = 0;  // rows with blocks so far (their O went through a V slot)
+    for (int k = 0; !failed; ++k) {
+      if (!warp_all(row_wait(k))) {
         failed = true;
         break;
       }
-      tc_fence_after();
-      // sv[4k + u]: row ra, key 8k + 2*t0 + u; sv[4k + 2 + u]: row rb, same key
-      uint32_t sv[64];
-      tmem_ld16x256b_x16(tS, sv);
-      tmem_wait_ld_regs64(sv);
-      const bool rag = it < 1024 ? ((ragged_bits[it >> 5] >> (it & 31)) & 1u)
-                                 : (kv_last < BN && col_idx[s0 + it] == nB - 1);
-      if (rag) {
+      const RowDesc* d = rdesc + (k & 1);
+      const int r = d->r;
+      if (r < 0) break;
+      const int s0 = d->s0, n = d->n;
+      const int bh = r / nB, q0 = (r - bh * nB) * BM;
+      const int qlen = min(BM, N - q0);
+      float mref_a = -INFINITY, mref_b = -INFINITY;  // reference maxima (log2 units)
+      float l_a = 0.f, l_b = 0.f;                    // this thread's share of the row sums
+      // Warps 4-7 start each row half a block behind warps 0-3 (they begin
+      // once S(1) is ready, one S MMA later than S(0)), so the two softmax
+      // warps of each SM sub-partition tend to be out of phase: one is in
+      // its exp2 stretch (MUFU-bound) while the other loads, reduces and
+      // stores.  (S(g + 4) cannot complete before these warps have produced
+      // P(g + 1), so the wait below sees the right phase of buffer g + 1.)
+#if DSA_SOFTMAX_LAG
+      if ((warp >> 2) == 1 && n > 1) {
+        const uint32_t g1 = g + 1;
+        if (!warp_all(mbar_wait(bar(kBarSFull + g1 % kSBufs), (g1 / kSBufs) & 1u))) {
+          failed = true;
+          break;
+        }
+      }
+#endif
+      for (int it = 0; it < n; ++it) {
+        const uint32_t gb = g + it;
+        const uint32_t b = gb % kSBufs;
+        const uint32_t tS = tmem + lane_off + 128u * b;
+        if (!warp_all(mbar_wait(bar(kBarSFull + b), (gb / kSBufs) & 1u))) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        // sv[4k + u]: row ra, key 8k + 2*t0 + u; sv[4k + 2 + u]: row rb, same key
+        uint32_t sv[64];
+        tmem_ld16x256b_x16(tS, sv);
+        tmem_wait_ld_regs64(sv);
+        const bool rag = it < 1024 ? ((d->ragged[it >> 5] >> (it & 31)) & 1u)
+                                   : (kv_last < BN && col_idx[s0 + it] == nB - 1);
+        if (rag) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
+          for (int kc = 0; kc < 16; ++kc)
 #pragma unroll
-          for (int u = 0; u < 2; ++u)
-            if (8 * k + 2 * t0 + u >= kv_last) {
-              sv[4 * k + u] = __float_as_uint(-INFINITY);
-              sv[4 * k + 2 + u] = __float_as_uint(-INFINITY);
+            for (int u = 0; u < 2; ++u)
+              if (8 * kc + 2 * t0 + u >= kv_last) {
+                sv[4 * kc + u] = __float_as_uint(-INFINITY);
+                sv[4 * kc + 2 + u] = __float_as_uint(-INFINITY);
+              }
+        }
+        // The exps run against the reference; the row maxima are computed
+        // only for the first block, or when a thread's partial row sums show
+        // the reference has fallen far below this block's maxima.
+        const uint64_t sc2 = pack_f32x2(scale_log2, scale_log2);
+        uint32_t pk[32];
+        float rs_a = 0.f, rs_b = 0.f;
+        auto exps = [&]() {
+          const uint64_t na2 = pack_f32x2(-mref_a, -mref_a), nb2 = pack_f32x2(-mref_b, -mref_b);
+          uint64_t rsa2[2] = {0ull, 0ull}, rsb2[2] = {0ull, 0ull};
+#pragma unroll
+          for (int kc = 0; kc < 16; ++kc) {
+            float a0, a1, b0, b1;
+            const uint64_t xa = fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * kc]), __uint_as_float(sv[4 * kc + 1])), sc2, na2);
+            const uint64_t xb = fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * kc + 2]), __uint_as_float(sv[4 * kc + 3])), sc2, nb2);
+            if (poly_chunk(kc, kPoly)) {
+              unpack_f32x2(exp2_poly_x2(xa), a0, a1);
+              unpack_f32x2(exp2_poly_x2(xb), b0, b1);
+            } else {
+              unpack_f32x2(xa, a0, a1);
+              unpack_f32x2(xb, b0, b1);
+              a0 = exp2_mufu(a0);
+              a1 = exp2_mufu(a1);
+              b0 = exp2_mufu(b0);
+              b1 = exp2_mufu(b1);
             }
-      }
-      // The exps run against the reference; the row maxima are computed only
-      // for the first block, or when a thread's partial row sums show the
-      // reference has fallen far below this block's maxima.
-      const uint64_t sc2 = pack_f32x2(scale_log2, scale_log2);
-      uint32_t pk[32];
-      float rs_a = 0.f, rs_b = 0.f;
-      auto exps = [&]() {
-        const uint64_t na2 = pack_f32x2(-mref_a, -mref_a), nb2 = pack_f32x2(-mref_b, -mref_b);
-        uint64_t rsa2[2] = {0ull, 0ull}, rsb2[2] = {0ull, 0ull};
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          float a0, a1, b0, b1;
-          const uint64_t xa = fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1])), sc2, na2);
-          const uint64_t xb = fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3])), sc2, nb2);
-          if (poly_chunk(k, kPoly)) {
-            unpack_f32x2(exp2_poly_x2(xa), a0, a1);
-            unpack_f32x2(exp2_poly_x2(xb), b0, b1);
-          } else {
-            unpack_f32x2(xa, a0, a1);
-            unpack_f32x2(xb, b0, b1);
-            a0 = exp2_mufu(a0);
-            a1 = exp2_mufu(a1);
-            b0 = exp2_mufu(b0);
-            b1 = exp2_mufu(b1);
+            rsa2[kc & 1] = add_f32x2(rsa2[kc & 1], pack_f32x2(a0, a1));
+            rsb2[kc & 1] = add_f32x2(rsb2[kc & 1], pack_f32x2(b0, b1));
+            const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1);
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(b0, b1);
+            pk[2 * kc] = *reinterpret_cast<const uint32_t*>(&ha);
+            pk[2 * kc + 1] = *reinterpret_cast<const uint32_t*>(&hb);
           }
-          rsa2[k & 1] = add_f32x2(rsa2[k & 1], pack_f32x2(a0, a1));
-          rsb2[k & 1] = add_f32x2(rsb2[k & 1], pack_f32x2(b0, b1));
-          const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1);
-          const __nv_bfloat162 hb = __floats2bfloat162_rn(b0, b1);
-          pk[2 * k] = *reinterpret_cast<const uint32_t*>(&ha);
-          pk[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&hb);
-        }
-        float u0, u1, u2, u3;
-        unpack_f32x2(add_f32x2(rsa2[0], rsa2[1]), u0, u1);
-        unpack_f32x2(add_f32x2(rsb2[0], rsb2[1]), u2, u3);
-        rs_a = u0 + u1;
-        rs_b = u2 + u3;
-      };
-      float alpha_a = 1.0f, alpha_b = 1.0f;
-      bool warp_need = false;
-      auto new_reference = [&]() {
-        float ma4[4], mb4[4];
+          float u0, u1, u2, u3;
+          unpack_f32x2(add_f32x2(rsa2[0], rsa2[1]), u0, u1);
+          unpack_f32x2(add_f32x2(rsb2[0], rsb2[1]), u2, u3);
+          rs_a = u0 + u1;
+          rs_b = u2 + u3;
+        };
+        float alpha_a = 1.0f, alpha_b = 1.0f;
+        bool warp_need = false;
+        auto new_reference = [&]() {
+          float ma4[4], mb4[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          ma4[u] = fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1]));
-          mb4[u] = fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]));
-        }
+          for (int u = 0; u < 4; ++u) {
+            ma4[u] = fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1]));
+            mb4[u] = fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]));
+          }
 #pragma unroll
-        for (int k = 4; k < 16; ++k) {
-          ma4[k & 3] = max3f(ma4[k & 3], __uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1]));
-          mb4[k & 3] = max3f(mb4[k & 3], __uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3]));
-        }
-        float ma = max3f(ma4[0], ma4[1], fmaxf(ma4[2], ma4[3]));
-        float mb = max3f(mb4[0], mb4[1], fmaxf(mb4[2], mb4[3]));
-        ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
-        ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-        const float xa = ma * scale_log2, xb = mb * scale_log2;
-        const bool need_a = xa > mref_a, need_b = xb > mref_b;
-        warp_need = __any_sync(0xffffffffu, need_a || need_b);
-        if (need_a) {
-          alpha_a = exp2f(mref_a - xa);  // 0 on the first block
-          l_a *= alpha_a;
-          mref_a = xa;
-        }
-        if (need_b) {
-          alpha_b = exp2f(mref_b - xb);
-          l_b *= alpha_b;
-          mref_b = xb;
-        }
-      };
-      if (it == 0) new_reference();
-      exps();
-      if (it > 0 && __any_sync(0xffffffffu, !(rs_a < kPMax) || !(rs_b < kPMax))) {
-        new_reference();
+          for (int kc = 4; kc < 16; ++kc) {
+            ma4[kc & 3] = max3f(ma4[kc & 3], __uint_as_float(sv[4 * kc]), __uint_as_float(sv[4 * kc + 1]));
+            mb4[kc & 3] = max3f(mb4[kc & 3], __uint_as_float(sv[4 * kc + 2]), __uint_as_float(sv[4 * kc + 3]));
+          }
+          float ma = max3f(ma4[0], ma4[1], fmaxf(ma4[2], ma4[3]));
+          float mb = max3f(mb4[0], mb4[1], fmaxf(mb4[2], mb4[3]));
+          ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+          mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+          ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+          mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+          const float xa = ma * scale_log2, xb = mb * scale_log2;
+          const bool need_a = xa > mref_a, need_b = xb > mref_b;
+          warp_need = __any_sync(0xffffffffu, need_a || need_b);
+          if (need_a) {
+            alpha_a = exp2f(mref_a - xa);  // 0 on the first block
+            l_a *= alpha_a;
+            mref_a = xa;
+          }
+          if (need_b) {
+            alpha_b = exp2f(mref_b - xb);
+            l_b *= alpha_b;
+            mref_b = xb;
+          }
+        };
+        if (it == 0) new_reference();
         exps();
-      }
-      tmem_st16x128b_x16(tS, pk);
-      if (warp_need && it > 0) {
-        // O holds the sum through block it-1; wait for PV(it-1), then move O to
-        // the new reference before PV(it) accumulates onto it
-        const int pb = (it - 1) % kStages;
-        if (!warp_all(mbar_wait(bar(kBarPVDone + pb), (uint32_t)((it - 1) / kStages) & 1u))) {
-          *abort_flag = 1;
-        } else {
+        if (it > 0 && __any_sync(0xffffffffu, !(rs_a < kPMax) || !(rs_b < kPMax))) {
+          new_reference();
+          exps();
+        }
+        tmem_st16x128b_x16(tS, pk);
+        if (warp_need && it > 0) {
+          // O holds the sum through block it-1; wait for PV(it-1), then move
+          // O to the new reference before PV(it) accumulates onto it
+          const uint32_t gp = gb - 1;
+          if (!warp_all(mbar_wait(bar(kBarPVDone + gp % kStages), (gp / kStages) & 1u))) {
+            failed = true;
+            break;
+          }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
@@ -517,110 +732,116 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             tmem_ld16x256b_x8(ta, o);
             tmem_wait_ld_regs(o);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * alpha_a);
-              o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * alpha_a);
-              o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * alpha_b);
-              o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * alpha_b);
+            for (int kc = 0; kc < 8; ++kc) {
+              o[4 * kc] = __float_as_uint(__uint_as_float(o[4 * kc]) * alpha_a);
+              o[4 * kc + 1] = __float_as_uint(__uint_as_float(o[4 * kc + 1]) * alpha_a);
+              o[4 * kc + 2] = __float_as_uint(__uint_as_float(o[4 * kc + 2]) * alpha_b);
+              o[4 * kc + 3] = __float_as_uint(__uint_as_float(o[4 * kc + 3]) * alpha_b);
             }
             tmem_st16x256b_x8(ta, o);
           }
         }
-      }
-      l_a += rs_a;
-      l_b += rs_b;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarPFull + b));
-      if (blk_lse != nullptr) {
-        // the block's share of each row's denominator: sum over the quad
-        float ta = rs_a + __shfl_xor_sync(0xffffffffu, rs_a, 1);
-        float tb = rs_b + __shfl_xor_sync(0xffffffffu, rs_b, 1);
-        ta += __shfl_xor_sync(0xffffffffu, ta, 2);
-        tb += __shfl_xor_sync(0xffffffffu, tb, 2);
-        if (t0 == 0) {
-          if (ra < qlen) blk_lse[(size_t)(s0 + it) * BN + ra] = (mref_a + lg2_mufu(ta)) * kLn2;
-          if (rb < qlen) blk_lse[(size_t)(s0 + it) * BN + rb] = (mref_b + lg2_mufu(tb)) * kLn2;
-        }
-      }
-    }
-
-    bool o_ok = false;  // this warp's rows of O are in shared memory
-    if (failed) {
-      *abort_flag = 1;
-      flag_error(err, kErrTimeout);
-    } else if (n > 0) {
-      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-      if (!warp_all(mbar_wait(bar(kBarPVDone + (n - 1) % kStages), (uint32_t)((n - 1) / kStages) & 1u))) {
-        *abort_flag = 1;
-        flag_error(err, kErrTimeout);
-      } else {
-        tc_fence_after();
-        const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
-        // D = 128: O / l as bf16 into the Q tile's shared memory (every MMA,
-        // and so every read of Q, is done), in the 128-byte-swizzled layout
-        // of the tensor map (16-byte chunk k of row r sits at chunk
-        // k ^ (r % 8)), for one TMA store below.  D = 64: straight to global
-        // memory (measured faster there).
-        uint8_t* sa = smem + L::kQ + ra * 128 + 4 * t0;
-        uint8_t* sb = smem + L::kQ + rb * 128 + 4 * t0;
-        __nv_bfloat16* ga = out + ((size_t)bh * N + q0 + ra) * D + 2 * t0;
-        __nv_bfloat16* gb = out + ((size_t)bh * N + q0 + rb) * D + 2 * t0;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t o[32];
-          tmem_ld16x256b_x8(tmem + lane_off + kTmemO + 64 * c, o);
-          tmem_wait_ld_regs(o);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const __nv_bfloat162 ha = __floats2bfloat162_rn(__uint_as_float(o[4 * k]) * inv_a,
-                                                            __uint_as_float(o[4 * k + 1]) * inv_a);
-            const __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[4 * k + 2]) * inv_b,
-                                                            __uint_as_float(o[4 * k + 3]) * inv_b);
-            if (kTmaStoreO) {
-              *reinterpret_cast<__nv_bfloat162*>(sa + c * L::kSub + ((k ^ (ra & 7)) << 4)) = ha;
-              *reinterpret_cast<__nv_bfloat162*>(sb + c * L::kSub + ((k ^ (rb & 7)) << 4)) = hb;
-            } else {
-              if (ra < qlen) *reinterpret_cast<__nv_bfloat162*>(ga + 64 * c + 8 * k) = ha;
-              if (rb < qlen) *reinterpret_cast<__nv_bfloat162*>(gb + 64 * c + 8 * k) = hb;
-            }
+        l_a += rs_a;
+        l_b += rs_b;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarPFull + b));
+        if (blk_lse != nullptr) {
+          // the block's share of each row's denominator: sum over the quad
+          float ta = rs_a + __shfl_xor_sync(0xffffffffu, rs_a, 1);
+          float tb = rs_b + __shfl_xor_sync(0xffffffffu, rs_b, 1);
+          ta += __shfl_xor_sync(0xffffffffu, ta, 2);
+          tb += __shfl_xor_sync(0xffffffffu, tb, 2);
+          if (t0 == 0) {
+            if (ra < qlen) blk_lse[(size_t)(s0 + it) * BN + ra] = (mref_a + lg2_mufu(ta)) * kLn2;
+            if (rb < qlen) blk_lse[(size_t)(s0 + it) * BN + rb] = (mref_b + lg2_mufu(tb)) * kLn2;
           }
         }
-        if (kTmaStoreO) fence_proxy_async_smem();
-        o_ok = true;
+      }
+      if (failed) break;
+
+      if (n > 0) {
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+        const uint32_t gl = g + n - 1;
+        if (!warp_all(mbar_wait(bar(kBarPVDone + gl % kStages), (gl / kStages) & 1u))) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
+        // O / l as bf16 into the V slot of the row's last block (PV of that
+        // block is done, so no MMA reads it any more), in the O tensor map's
+        // 128-byte-swizzled layout: 16-byte chunk k of row r of each 64-column
+        // sub-tile sits at chunk k ^ (r % 8).  The V loader stores the tile
+        // with TMA.  This warp's reads of O are done (tcgen05.wait::ld)
+        // before it writes the next row's first P, which is what lets that
+        // row's first PV overwrite O.  The four threads of a quad swap their
+        // packed pairs so that each holds 8 consecutive columns of one row
+        // and writes them as one 16-byte chunk.
+        uint32_t o[64];  // o[4k + u]: row ra, column 8k + 2*t0 + u; o[4k + 2 + u]: row rb
+        if constexpr (D == 128) {
+          tmem_ld16x256b_x16(tmem + lane_off + kTmemO, o);
+          tmem_wait_ld_regs64(o);
+        } else {
+          uint32_t(&o32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+          tmem_ld16x256b_x8(tmem + lane_off + kTmemO, o32);
+          tmem_wait_ld_regs(o32);
+        }
+        uint8_t* stage = smem + L::kV + (gl % kStages) * kTileBytes;
+#pragma unroll
+        for (int h = 0; h < D / 32; ++h) {  // chunks 4h .. 4h+3 (columns 32h .. 32h+31)
+          uint32_t xa[4], xb[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int kc = 4 * h + j;
+            const __nv_bfloat162 ha = __floats2bfloat162_rn(__uint_as_float(o[4 * kc]) * inv_a,
+                                                            __uint_as_float(o[4 * kc + 1]) * inv_a);
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[4 * kc + 2]) * inv_b,
+                                                            __uint_as_float(o[4 * kc + 3]) * inv_b);
+            xa[j] = *reinterpret_cast<const uint32_t*>(&ha);
+            xb[j] = *reinterpret_cast<const uint32_t*>(&hb);
+          }
+          quad_transpose(xa, t0);  // xa[u]: columns 8(4h + t0) + 2u, +1
+          quad_transpose(xb, t0);
+          const int ch = 4 * h + t0, c = ch >> 3, kk = ch & 7;
+          *reinterpret_cast<uint4*>(stage + c * L::kSub + ra * 128 + ((kk ^ (ra & 7)) << 4)) =
+              make_uint4(xa[0], xa[1], xa[2], xa[3]);
+          *reinterpret_cast<uint4*>(stage + c * L::kSub + rb * 128 + ((kk ^ (rb & 7)) << 4)) =
+              make_uint4(xb[0], xb[1], xb[2], xb[3]);
+        }
+        fence_proxy_async_smem();  // visible to the TMA store
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarOStaged + orows % kStages));
+        ++orows;
         if (t0 == 0 && lse != nullptr) {
           if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
           if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
         }
-      }
-    } else {
-      const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
+      } else {
+        __nv_bfloat16* ra_out = out + ((size_t)bh * N + q0 + ra) * D;
+        __nv_bfloat16* rb_out = out + ((size_t)bh * N + q0 + rb) * D;
 #pragma unroll
-      for (int k = 0; k < D / 8; ++k) {
-        if (ra < qlen) *reinterpret_cast<__nv_bfloat162*>(out + ((size_t)bh * N + q0 + ra) * D + 8 * k + 2 * t0) = z;
-        if (rb < qlen) *reinterpret_cast<__nv_bfloat162*>(out + ((size_t)bh * N + q0 + rb) * D + 8 * k + 2 * t0) = z;
+        for (int h = 0; h < D / 32; ++h) {
+          if (ra < qlen) *reinterpret_cast<uint4*>(ra_out + 8 * (4 * h + t0)) = make_uint4(0u, 0u, 0u, 0u);
+          if (rb < qlen) *reinterpret_cast<uint4*>(rb_out + 8 * (4 * h + t0)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (t0 == 0 && lse != nullptr) {
+          if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = -INFINITY;
+          if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = -INFINITY;
+        }
       }
-      if (t0 == 0 && lse != nullptr) {
-        if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = -INFINITY;
-        if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = -INFINITY;
-      }
+      // done with this row's descriptor (its ragged marks)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarRowFree + (k & 1)));
+      g += n;
     }
-    if (kTmaStoreO && n > 0) {
-      // Every softmax warp arrives here, the ones that gave up too, so none
-      // waits alone; then one thread stores the O tile with TMA (rows past N
-      // fall outside the tensor and are not written) and waits until the
-      // copy has read shared memory.
-      const bool any_fail = named_bar_or(1, kSoftmaxThreads, !o_ok);
-      if (!any_fail && tid == 0) {
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, sQ + c * L::kSub, c * 64, q0, bh);
-        tma_store_commit();
-        tma_store_wait_read();
-      }
+    if (failed) {
+      *abort_flag = 1;
+      if (lane == 0) flag_error(err, kErrTimeout);
     }
   }
 
@@ -629,18 +850,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (*abort_flag) {
     // A role gave up: copies and MMAs may still be in flight.  Let every one
     // of them finish (bounded) before shared and tensor memory are released.
-    if (warp == kMmaWarp && n > 0) {
+    if (warp == kMmaWarp && had_rows) {
       if (lane == 0) {
         mma_commit(bar(kBarDrain));  // arrives once all MMAs issued so far are done
         mbar_wait(bar(kBarDrain), 0u);
       }
       __syncwarp();
-    } else if (warp == kLoadWarp && lane == 0 && n > 0) {
-      for (int b = k_issued - kStages > 0 ? k_issued - kStages : 0; b < k_issued; ++b)
-        mbar_wait(bar(kBarKFull + b % kStages), (uint32_t)(b / kStages) & 1u);
-      for (int b = v_issued - kStages > 0 ? v_issued - kStages : 0; b < v_issued; ++b)
-        mbar_wait(bar(kBarVFull + b % kStages), (uint32_t)(b / kStages) & 1u);
-      mbar_wait(bar(kBarQ), 0u);
+    } else if (warp == kKLoadWarp && lane == 0) {
+      for (uint32_t b = k_issued > kStages ? k_issued - kStages : 0; b < k_issued; ++b)
+        mbar_wait(bar(kBarKFull + b % kStages), (b / kStages) & 1u);
+      if (q_issued > 0) mbar_wait(bar(kBarQ), (q_issued - 1) & 1u);
+    } else if (warp == kVLoadWarp && lane == 0) {
+      for (uint32_t b = v_issued > kStages ? v_issued - kStages : 0; b < v_issued; ++b)
+        mbar_wait(bar(kBarVFull + b % kStages), (b / kStages) & 1u);
     }
     tc_fence_before();
     __syncthreads();
@@ -649,7 +871,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  // The last CTA to finish resets the launch's ticket counter for the next
+  // launch that uses it (every CTA has drawn its last ticket by now).
+  if (tid == 0 && atomicAdd(&tickets[1], 1u) == gridDim.x - 1) {
+    atomicExch(&tickets[0], 0u);
+    atomicExch(&tickets[1], 0u);
+  }
 }
+
 
 // cuTensorMapEncodeTiled, looked up once through the runtime (no -lcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -685,19 +914,23 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int D) {
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mo, int BH,
-                     int N, float scale, const int32_t* row_ptr, const int32_t* col_idx,
-                     void* out, float* lse, float* blk_lse, unsigned* err, cudaStream_t s) {
+                     const CUtensorMap& mo, int BH, int N, float scale, const int32_t* row_ptr, const int32_t* col_idx,
+                     void* out, float* lse, float* blk_lse, unsigned* tickets, int num_sms,
+                     unsigned* err, cudaStream_t s) {
   const int nB = ceil_div(N, BN);
   const int rows = BH * nB;
+  if (rows == 0) return cudaSuccess;
   const int smem = SmemLayout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
-  attn_fwd_sm100_kernel<D><<<rows, kThreads, smem, s>>>(
-      mq, mk, mv, mo, N, nB, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out), lse,
-      blk_lse, err);
+  // one CTA per SM (384 threads at up to 168 registers fill an SM's register
+  // file, so no second CTA fits beside one)
+  const int grid = rows < num_sms ? rows : num_sms;
+  attn_fwd_sm100_kernel<D><<<grid, kThreads, smem, s>>>(
+      mq, mk, mv, mo, N, nB, rows, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out),
+      lse, blk_lse, tickets, err);
   return cudaGetLastError();
 }
 
@@ -706,15 +939,19 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int BH, int N,
                               int D, float scale, const int32_t* row_ptr,
                               const int32_t* col_idx, void* out, float* lse, float* blk_lse,
-                              unsigned* err, cudaStream_t s, const char** why) {
+                              unsigned* tickets, int num_sms, unsigned* err, cudaStream_t s,
+                              const char** why) {
   CUtensorMap mq, mk, mv, mo;
   if (!make_tile_map(&mq, q, BH, N, D) || !make_tile_map(&mk, k, BH, N, D) ||
       !make_tile_map(&mv, v, BH, N, D) || !make_tile_map(&mo, out, BH, N, D)) {
     if (why) *why = "cuTensorMapEncodeTiled failed or is unavailable";
     return cudaErrorInvalidValue;
   }
-  if (D == 64) return launch_d<64>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, err, s);
-  return launch_d<128>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, err, s);
+  if (D == 64)
+    return launch_d<64>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, tickets,
+                        num_sms, err, s);
+  return launch_d<128>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, tickets,
+                       num_sms, err, s);
 }
 
 }  // namespace dsa

@@ -52,11 +52,13 @@ cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, bool b
                              int BH, int N, int D, int block, float scale,
                              const int32_t* row_ptr, const int32_t* col_idx, void* out,
                              float* lse, float* blk_lse, unsigned* err, cudaStream_t s);
+// tickets: two zeroed words of device memory that no concurrent launch uses
+// (the kernel leaves them zeroed); num_sms: the device's SM count.
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int BH,
                               int N, int D, float scale, const int32_t* row_ptr,
                               const int32_t* col_idx, void* out, float* lse,
-                              float* blk_lse, unsigned* err, cudaStream_t s,
-                              const char** why);
+                              float* blk_lse, unsigned* tickets, int num_sms,
+                              unsigned* err, cudaStream_t s, const char** why);
 cudaError_t launch_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx,
                                  const float* mass, int rows, int nB, float* probs,
                                  unsigned* err, cudaStream_t s);

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -27,6 +28,14 @@ thread_local std::string g_last_error;
 
 // Device-side error word shared by all kernels of the library.
 __device__ unsigned g_device_error;
+
+// Ticket counters of the tensor-core attention kernel, which hands its rows
+// to persistent CTAs dynamically: each launch takes one pair (next row,
+// finished CTAs), in rotation, and its last CTA zeroes the pair again.
+// Launches that overlap in time use different pairs while fewer than
+// kTicketPairs launches lie between them.
+constexpr unsigned kTicketPairs = 4096;
+__device__ unsigned g_attn_tickets[2 * kTicketPairs];
 
 constexpr int kMaxDevices = 64;
 
@@ -49,6 +58,9 @@ struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
   unsigned* err_word = nullptr;
+  unsigned* tickets = nullptr;    // g_attn_tickets on this device
+  int num_sms = 0;
+  std::atomic<unsigned> next_pair{0};
 };
 
 std::mutex g_dev_mutex;
@@ -73,6 +85,11 @@ dsa_status device_info(DeviceInfo** out) {
       e = cudaGetSymbolAddress(&p, g_device_error);
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
       d.err_word = static_cast<unsigned*>(p);
+      e = cudaGetSymbolAddress(&p, g_attn_tickets);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+      d.tickets = static_cast<unsigned*>(p);
+      e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     }
     d.init = true;
   }
@@ -257,8 +274,9 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
   cudaError_t e;
   if (dt == DSA_BF16 && block == 128 && N >= 128) {
     const char* why = nullptr;
+    const unsigned pair = dev->next_pair.fetch_add(1u) % kTicketPairs;
     e = dsa::launch_attn_sm100(q, k, v, BH, N, D, scale, row_ptr, col_idx, out, lse, blk_lse,
-                               dev->err_word, s, &why);
+                               dev->tickets + 2 * pair, dev->num_sms, dev->err_word, s, &why);
     if (e != cudaSuccess && why) return fail(DSA_ERR_CUDA, "attn_fwd: %s", why);
   } else {
     e = dsa::launch_attn_simt(q, k, v, dt == DSA_BF16, BH, N, D, block, scale, row_ptr, col_idx,

@@ -186,6 +186,17 @@ dsa_status dsa_select_topp(const float* probs, int rows, int nB, float p,
  * A row with no blocks gives O = 0.  bf16 runs on tcgen05 tensor cores with
  * fp32 accumulation; fp32 (and block 64) runs on an exact-fp32 CUDA-core
  * path.
+ * Scheduling (bf16, block 128): one persistent CTA per SM takes rows from a
+ * ticket counter in device memory that the library keeps per device (4,096
+ * counters used in rotation, one per launch; the launch's last CTA zeroes its
+ * counter again), so rows of skewed length are balanced dynamically (DSV
+ * abstract).  Launches that run at the same time, on any streams, use
+ * different counters while fewer than 4,096 launches lie between them; a
+ * captured CUDA graph replays its launch with the counter of its capture.
+ * Errors: a malformed row (column index outside [0, nB), decreasing row_ptr)
+ * sets the device error word and is written as an empty row; a device wait
+ * that runs out (1 s) sets the error word and leaves the rows that the
+ * affected CTA had not finished unwritten.  dsa_device_status reports both.
  */
 dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype dt,
                         int B, int H, int N, int D, int block, float scale,
