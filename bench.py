@@ -47,8 +47,8 @@ ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn
 # prefix of attn_sm100.cu at capture time (scaled to the full workload when
 # the capture ran a smaller case); stale entries are ignored.
 ATTN_TRAFFIC = {
-    # 8-head Wan2.1-like capture: 551.8 MB read + 501.9 MB written, x5 heads
-    "0dce65c8e57a2f3e": int((551810304 + 501890304) * 5),
+    # 8-head Wan2.1-like capture: 662.6 MB read + 501.6 MB written, x5 heads
+    "3400822f2e6fef1e": int((662567680 + 501644544) * 5),
 }
 
 
