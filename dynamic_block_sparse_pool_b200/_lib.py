@@ -38,6 +38,7 @@ SIGNATURES = {
     "dsa_permute_tokens": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp]),
     "dsa_select_topp_static": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]),
     "dsa_selftest_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),
+    "dsa_selftest_exp2_poly": (_i, [_vp, _vp, _i, _vp]),
     "dsa_device_status": (_i, [_vp]),
     "dsa_last_error": (ctypes.c_char_p, []),
     "dsa_version": (_i, []),

@@ -179,41 +179,6 @@ __host__ __device__ constexpr bool poly_chunk(int k, int kPoly) {
   return (k + 1) * kPoly / 16 != k * kPoly / 16;
 }
 
-// 2^x for a pair of fp32 values on the FMA pipe.  Range reduction in the
-// manner of Cody and Waite for base 2: x = j + r with j = round(x), taken by
-// adding the shifter 1.5 * 2^23 (the sum keeps j in its low mantissa bits)
-// and r = x - j in [-0.5, 0.5]; 2^r by the degree-4 polynomial of least
-// maximum relative error on [-0.5, 0.5] (Remez exchange, error 2.6e-6, 2.7e-6
-// when evaluated in fp32); 2^j by adding j to the exponent field of 2^r.  x is
-// clamped to [-126, 127] first, so the exponent stays in range: results
-// below 2^-126 come out as about 2^-126 instead of 0, and anything that
-// would overflow comes out at or above 2^126.5.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99999928474426270f, c1 = 0.69312179088592529f,
-                  c2 = 0.24024743318367004f, c3 = 0.055917859077453613f,
-                  c4 = 0.0095701022073626518f;
-  float x0, x1;
-  unpack_f32x2(x2, x0, x1);
-  x0 = fminf(fmaxf(x0, -126.0f), 127.0f);
-  x1 = fminf(fmaxf(x1, -126.0f), 127.0f);
-  const uint64_t xc = pack_f32x2(x0, x1);
-  const uint64_t t = add_f32x2(xc, pack_f32x2(kShift, kShift));     // shifter + j
-  const uint64_t j = add_f32x2(t, pack_f32x2(-kShift, -kShift));    // j, exactly
-  const uint64_t r = fma_f32x2(j, pack_f32x2(-1.0f, -1.0f), xc);    // x - j, exactly
-  uint64_t p = fma_f32x2(pack_f32x2(c4, c4), r, pack_f32x2(c3, c3));
-  p = fma_f32x2(p, r, pack_f32x2(c2, c2));
-  p = fma_f32x2(p, r, pack_f32x2(c1, c1));
-  p = fma_f32x2(p, r, pack_f32x2(c0, c0));
-  float t0, t1, p0, p1;
-  unpack_f32x2(t, t0, t1);
-  unpack_f32x2(p, p0, p1);
-  // (shifter + j) << 23 leaves j << 23 (the shifter's bits shift out)
-  const uint32_t e0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
-  const uint32_t e1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
-  return pack_f32x2(__uint_as_float(e0), __uint_as_float(e1));
-}
-
 // 4 x 4 transpose of 32-bit words across the four threads of a quad (lanes
 // 4q .. 4q+3, t = lane % 4): afterwards x[u] holds what thread u held in
 // x[t].  Two butterfly steps: transpose the 2 x 2 blocks (partner t ^ 1),

@@ -86,6 +86,7 @@ cudaError_t launch_attn_bwd_sm100(const void* q, const void* k, const void* v, c
                                   void* dv, unsigned* err, cudaStream_t s);
 // One CTA that waits on an mbarrier nobody arrives at, with the given limit.
 cudaError_t launch_wait_timeout(unsigned long long limit_ns, unsigned* err, cudaStream_t s);
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_block_mass(const float* lse, const float* blk_lse, int BH, int N,
                               int block, const int32_t* row_ptr, float* mass,
                               cudaStream_t s);

@@ -431,6 +431,20 @@ dsa_status dsa_selftest_wait_timeout(unsigned long long limit_ns, void* stream) 
   return DSA_OK;
 }
 
+dsa_status dsa_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  g_last_error.clear();
+  if (n < 0) return fail(DSA_ERR_INVALID_ARG, "n must be >= 0 (got %d)", n);
+  if (n > 0 && (x == nullptr || y == nullptr)) return fail(DSA_ERR_INVALID_ARG, "x and y must not be null");
+  if (!aligned(x, 4) || !aligned(y, 4)) return fail(DSA_ERR_INVALID_ARG, "x and y must be 4-byte aligned");
+  DeviceInfo* dev = nullptr;
+  dsa_status st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  if (n == 0) return DSA_OK;
+  cudaError_t e = dsa::launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "exp2_poly launch");
+  return DSA_OK;
+}
+
 dsa_status dsa_device_status(void* stream) {
   g_last_error.clear();
   DeviceInfo* dev = nullptr;

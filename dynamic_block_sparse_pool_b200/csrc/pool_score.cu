@@ -14,9 +14,10 @@
 //   the fine row softmax back into block rows (token-weighted over query
 //   sub-blocks, summed over key sub-blocks).
 // Kernel 2 (block_scores): one CTA per (64 query-block rows, head): a
-//   register-tiled fp32 product of the 64 pooled queries with double-buffered
-//   tiles of 64 pooled keys (cp.async), scaled scores written to P with a
-//   running max and sum per row, then P normalised in place from L2.
+//   register-tiled fp32 product of the 64 pooled queries with tiles of 64
+//   pooled keys (cp.async; one tile buffer and three CTAs per SM), scaled
+//   scores written to P with a running max and sum per row, then P
+//   normalised in place from L2.
 #include "common.cuh"
 
 namespace dsa {
@@ -62,6 +63,15 @@ pool_means_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int n
 }
 
 constexpr int kTile = 64;  // query-block rows per CTA and key blocks per score tile
+// Key tiles in shared memory: with one (76 KB per CTA, 80 registers) three
+// CTAs fit on an SM, and the other two hide each one's tile loads; with two
+// (double buffering, 110 KB) only two fit, and a launch over 40 heads (400
+// CTAs) takes two waves of 296 slots.
+#ifndef DSA_SCORE_KBUFS
+#define DSA_SCORE_KBUFS 1
+#endif
+constexpr int kKBufs = DSA_SCORE_KBUFS;
+constexpr int kScoreCtasPerSm = kKBufs == 1 ? 3 : 2;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
@@ -82,7 +92,7 @@ struct ScoreSmem {
   static constexpr int kStride = D + 4;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile * kStride;          // floats
-  static constexpr int kBits = kK + 2 * kTile * kStride;   // floats -> uint32 [64][32]
+  static constexpr int kBits = kK + kKBufs * kTile * kStride;  // floats -> uint32 [64][32]
   static constexpr int kStat = kBits + kTile * 32;         // float2 [64]
   static constexpr size_t kBytes = sizeof(float) * (size_t)(kStat + 2 * kTile);
 };
@@ -112,7 +122,7 @@ __device__ __forceinline__ void stage_rows(float* dst, const float* src, int fir
 //   Pass 2: one warp per row rewrites P as exp(s - max) / sum (reads hit L2:
 //     the CTA wrote them just before).  Non-candidates and empty rows get 0.
 template <int D>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, kScoreCtasPerSm)
 block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                     int nB, float scale, const int32_t* __restrict__ cand_row_ptr,
                     const int32_t* __restrict__ cand_col, float* __restrict__ probs,
@@ -180,13 +190,17 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
   int t = live ? __ffs(live) - 1 : n_tiles;
   if (t < n_tiles) stage_rows<D>(ks, khead, t * kTile, min(kTile, nB - t * kTile), tid);
   cp_async_commit();
-  for (int buf = 0; t < n_tiles; buf ^= 1) {
+  for (int buf = 0; t < n_tiles; buf = kKBufs == 2 ? buf ^ 1 : 0) {
     live &= ~(1u << t);
     const int tn = live ? __ffs(live) - 1 : n_tiles;
-    if (tn < n_tiles)
-      stage_rows<D>(ks + (buf ^ 1) * kTile * S, khead, tn * kTile, min(kTile, nB - tn * kTile), tid);
-    cp_async_commit();
-    cp_async_wait<1>();
+    if (kKBufs == 2) {
+      if (tn < n_tiles)
+        stage_rows<D>(ks + (buf ^ 1) * kTile * S, khead, tn * kTile, min(kTile, nB - tn * kTile), tid);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
 
     const float* kt = ks + buf * kTile * S;
@@ -237,7 +251,11 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
       for (int c = 0; c < 4; ++c)
         if (ok[c]) run_s[a] += expf(x[c] - run_m[a]);
     }
-    __syncthreads();  // this buffer is refilled two tiles later
+    __syncthreads();  // every read of this buffer is done; it is refilled next
+    if (kKBufs == 1) {
+      if (tn < n_tiles) stage_rows<D>(ks, khead, tn * kTile, min(kTile, nB - tn * kTile), tid);
+      cp_async_commit();
+    }
     t = tn;
   }
   cp_async_wait<0>();

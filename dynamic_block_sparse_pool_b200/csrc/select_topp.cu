@@ -234,13 +234,25 @@ select_kernel(const float* __restrict__ probs, int rows, int nB, float p,
     if (cs < 0 || ce < cs) {
       if (lane == 0) flag_error(err, kErrRowPtr);
     } else {
-      for (int e = cs + lane; e < ce; e += 32) {
-        const int j = cand_col[e];
-        if (j < 0 || j >= nB) {
-          flag_error(err, kErrCsrIndex);
-          continue;
+      // four independent index loads per lane in flight, then the marks
+      constexpr int kU = 4;
+      for (int e0 = cs + lane; e0 < ce; e0 += 32 * kU) {
+        int jj[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int e = e0 + 32 * u;
+          jj[u] = e < ce ? cand_col[e] : 0;
         }
-        atomicOr(&cbits[j >> 5], 1u << (j & 31));
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          if (e0 + 32 * u >= ce) continue;  // past the row's end
+          const int j = jj[u];
+          if (j < 0 || j >= nB) {
+            flag_error(err, kErrCsrIndex);
+            continue;
+          }
+          atomicOr(&cbits[j >> 5], 1u << (j & 31));
+        }
       }
     }
     __syncwarp();

@@ -274,6 +274,17 @@ def selftest_wait_timeout(limit_ns: int = 1_000_000, device: Optional[torch.devi
     check(lib().dsa_selftest_wait_timeout(int(limit_ns), s), "dsa_selftest_wait_timeout")
 
 
+def selftest_exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """2^x by the attention softmax's FMA-pipe exponential (fp32 CUDA tensor)."""
+    if not (x.is_cuda and x.dtype == torch.float32):
+        raise ValueError("x must be a float32 CUDA tensor")
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    s = torch.cuda.current_stream(x.device).cuda_stream
+    check(lib().dsa_selftest_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), s), "dsa_selftest_exp2_poly")
+    return y
+
+
 def device_status(device: Optional[torch.device] = None) -> None:
     """Synchronises the current stream and raises DSAError if a kernel flagged bad input."""
     s = torch.cuda.current_stream(device).cuda_stream

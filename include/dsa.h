@@ -16,6 +16,7 @@
  *   dsa_attn_bwd     gradients of the attention for a fixed mask.
  *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
  *                    exact attention weights (the next mask of a schedule).
+ *   dsa_selftest_wait_timeout, dsa_selftest_exp2_poly  self-tests.
  *   dsa_hilbert_order, dsa_gilbert_order, dsa_permute_tokens  token
  *                    reordering along a 3-D Hilbert curve (the enclosing
  *                    cube's, or one generalised to the grid's own box) before
@@ -378,6 +379,25 @@ dsa_status dsa_select_topp_static(const float* probs, int rows, int nB, float p,
  * Errors: DSA_ERR_INVALID_ARG for a limit outside that range.
  */
 dsa_status dsa_selftest_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/*
+ * Self-test of the attention softmax's FMA-pipe exponential (a build-time
+ * option, off by default: exponentials then all run on the MUFU).
+ * (No counterpart in the papers: GSRS's abstract computes the exact softmax
+ * weights; this checks the arithmetic that may produce them.)
+ * y[i] = 2^x[i] by the same device function the attention kernel uses:
+ * Cody-Waite reduction x = j + r, j = round(x), |r| <= 1/2; 2^r by a
+ * degree-4 polynomial of least maximum relative error on [-1/2, 1/2]
+ * (Remez exchange); 2^j added to the exponent field.  x is first clamped to
+ * [-126, 127].  Relative error below 3e-6 over that range (about 25 units in
+ * the last place of fp32, far below the 2^-9 of the bf16 P it feeds).
+ *
+ *   x, y   device, fp32 [n], 4-byte aligned; y is written, x is not.
+ *   n      >= 0.
+ * Asynchronous on `stream`.  Errors: DSA_ERR_INVALID_ARG for n < 0 or a null
+ * or misaligned pointer with n > 0.
+ */
+dsa_status dsa_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device-side

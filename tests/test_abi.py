@@ -23,7 +23,7 @@ def lib():
 def declared_symbols():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_four_pipeline_calls():
@@ -37,7 +37,7 @@ def declared_prototypes():
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     protos = {}
     for ret, name, params in re.findall(
-            r"^\s*((?:const\s+)?[a-z_0-9]+\s*\**)\s*(dsa_[a-z_]+)\s*\(([^)]*)\)\s*;",
+            r"^\s*((?:const\s+)?[a-z_0-9]+\s*\**)\s*(dsa_[a-z0-9_]+)\s*\(([^)]*)\)\s*;",
             text, flags=re.M):
         params = " ".join(params.split())
         types = [] if params in ("", "void") else [
