@@ -731,13 +731,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
         l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+        // lse and 1/l need only the row sums: they are done while the last
+        // PV runs
+        if (t0 == 0 && lse != nullptr) {
+          if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
+          if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
+        }
+        const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
         const uint32_t gl = g + n - 1;
         if (!warp_all(mbar_wait(bar(kBarPVDone + gl % kStages), (gl / kStages) & 1u))) {
           failed = true;
           break;
         }
         tc_fence_after();
-        const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
         // O / l as bf16 into the V slot of the row's last block (PV of that
         // block is done, so no MMA reads it any more), in the O tensor map's
         // 128-byte-swizzled layout: 16-byte chunk k of row r of each 64-column
@@ -782,10 +788,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kBarOStaged + orows % kStages));
         ++orows;
-        if (t0 == 0 && lse != nullptr) {
-          if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
-          if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
-        }
       } else {
         __nv_bfloat16* ra_out = out + ((size_t)bh * N + q0 + ra) * D;
         __nv_bfloat16* rb_out = out + ((size_t)bh * N + q0 + rb) * D;

@@ -159,13 +159,25 @@ block_scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kb
         if (lane == 0) flag_error(err, kErrRowPtr);
         continue;
       }
-      for (int e = cs + lane; e < ce; e += 32) {
-        const int j = cand_col[e];
-        if (j < 0 || j >= nB) {
-          flag_error(err, kErrCsrIndex);
-          continue;
+      // four independent index loads per lane in flight, then the marks
+      constexpr int kU = 4;
+      for (int e0 = cs + lane; e0 < ce; e0 += 32 * kU) {
+        int jj[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int e = e0 + 32 * u;
+          jj[u] = e < ce ? cand_col[e] : 0;
         }
-        atomicOr(&cbits[rr * 32 + (j >> 5)], 1u << (j & 31));
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          if (e0 + 32 * u >= ce) continue;  // past the row's end
+          const int j = jj[u];
+          if (j < 0 || j >= nB) {
+            flag_error(err, kErrCsrIndex);
+            continue;
+          }
+          atomicOr(&cbits[rr * 32 + (j >> 5)], 1u << (j & 31));
+        }
       }
     }
     __syncthreads();
