@@ -47,8 +47,8 @@ ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn
 # prefix of attn_sm100.cu at capture time (scaled to the full workload when
 # the capture ran a smaller case); stale entries are ignored.
 ATTN_TRAFFIC = {
-    # 8-head Wan2.1-like capture: 662.6 MB read + 501.6 MB written, x5 heads
-    "3400822f2e6fef1e": int((662567680 + 501644544) * 5),
+    # 8-head Wan2.1-like capture: 642.1 MB read + 500.2 MB written, x5 heads
+    "0b6b551a47819654": int((642087936 + 500244480) * 5),
 }
 
 
@@ -709,8 +709,9 @@ def main():
         }
         del rp_all, col_all
 
-    # end to end through the public host-buffer call: pinned Q, K, V in, O out,
-    # with the PCIe copies of one chunk of heads overlapping another's compute
+    # end to end through the library's host-buffer call (dsa_sparse_attention_host):
+    # pinned Q, K, V in, O out, with the PCIe copies of one chunk of heads
+    # overlapping another's compute
     if not args.no_e2e:
         from dynamic_block_sparse_pool_b200.pipeline import HostPipeline
         qh, kh, vh = q_c.pin_memory(), k_c.pin_memory(), v_c.pin_memory()
@@ -727,7 +728,8 @@ def main():
         torch.cuda.synchronize(dev)
         ms_e2e = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ee[1:]) / ke, world)
         line["e2e"] = {"value": total_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-                       "ms_per_step": ms_e2e, "api": "pipeline.HostPipeline.run",
+                       "ms_per_step": ms_e2e,
+                       "api": "dsa_sparse_attention_host (C ABI, host buffers)",
                        "chunk_heads": pipe.chunk,
                        "h2d_bytes_per_step": pipe.h2d_bytes(),
                        "d2h_bytes_per_step": pipe.d2h_bytes()}

@@ -39,6 +39,9 @@ SIGNATURES = {
     "dsa_select_topp_static": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]),
     "dsa_selftest_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),
     "dsa_selftest_exp2_poly": (_i, [_vp, _vp, _i, _vp]),
+    "dsa_sparse_attention_host": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _i, _vp, _vp,
+                                       _sz, _vp]),
+    "dsa_host_pipeline_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "dsa_device_status": (_i, [_vp]),
     "dsa_last_error": (ctypes.c_char_p, []),
     "dsa_version": (_i, []),

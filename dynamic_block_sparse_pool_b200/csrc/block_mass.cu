@@ -8,8 +8,8 @@
 // where blk_lse[s, t] is the log of the block's share of the softmax
 // denominator and lse_t the log of the whole denominator (both written by
 // the attention kernel).  One CTA per CSR row; each of its 8 warps keeps the
-// row's lse values in registers and reduces every 8th slot, reading that
-// slot's block-size run of blk_lse once, coalesced.
+// row's lse values in registers and reduces every 8th slot, two at a time,
+// reading each slot's block-size run of blk_lse once, coalesced.
 //
 // mass_to_probs scatters those masses back into dense rows, so that a Top-p
 // selection can run on exact attention weights (GSRS abstract: Top-p
@@ -27,30 +27,51 @@ block_mass_kernel(const float* __restrict__ lse, const float* __restrict__ blk, 
   constexpr int PER = BS / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x;
-  const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
-  if (s1 <= s0) return;
   const int bh = r / nB, i = r - bh * nB;
   const int q0 = i * BS;
   const int qlen = min(BS, N - q0);
+  // the row's lse values load together with its row_ptr entries (they
+  // depend on the row index only)
   float lv[PER];
 #pragma unroll
   for (int m = 0; m < PER; ++m) {
     const int t = lane + 32 * m;
     lv[m] = t < qlen ? lse[(size_t)bh * N + q0 + t] : 0.f;
   }
+  const int s0 = row_ptr[r], s1 = row_ptr[r + 1];
+  if (s1 <= s0) return;
   const float inv = 1.0f / (float)qlen;
-  // the row's slots are spread over the CTA's 8 warps
-  for (int s = s0 + warp; s < s1; s += 8) {
-    const float* b = blk + (size_t)s * BS;
-    float acc = 0.f;
+  // the row's slots are spread over the CTA's 8 warps, two slots per step
+  // (2 * PER loads per lane in flight)
+  for (int s = s0 + warp; s < s1; s += 16) {
+    const bool two = s + 8 < s1;
+    const float* b0 = blk + (size_t)s * BS;
+    const float* b1 = blk + (size_t)(two ? s + 8 : s) * BS;
+    float x0[PER], x1[PER];
 #pragma unroll
     for (int m = 0; m < PER; ++m) {
       const int t = lane + 32 * m;
-      if (t < qlen) acc += expf(b[t] - lv[m]);
+      x0[m] = t < qlen ? b0[t] : 0.f;
+      x1[m] = t < qlen ? b1[t] : 0.f;
+    }
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < PER; ++m) {
+      const int t = lane + 32 * m;
+      if (t < qlen) {
+        acc0 += expf(x0[m] - lv[m]);
+        acc1 += expf(x1[m] - lv[m]);
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) mass[s] = acc * inv;
+    for (int o = 16; o > 0; o >>= 1) {
+      acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+      acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+    }
+    if (lane == 0) {
+      mass[s] = acc0 * inv;
+      if (two) mass[s + 8] = acc1 * inv;
+    }
   }
 }
 

@@ -123,6 +123,70 @@ bool cand_ok(const int32_t* rp, const int32_t* col) { return (rp == nullptr) == 
 
 size_t pool_ws_bytes(long long BH, long long nB, int D) { return (size_t)(2 * BH * nB * D) * sizeof(float); }
 size_t select_ws_bytes(long long rows) { return (size_t)(rows * 33) * sizeof(uint32_t); }
+
+// ---- host-buffer pipeline (dsa_sparse_attention_host) ----
+
+// Byte offsets of one chunk's device buffers inside a pipeline slot, each
+// 256-byte aligned; `bytes` is the slot's size.
+struct HostSlot {
+  size_t q, k, v, out, lse, probs, ws_pool, ws_sel, row_ptr, col_idx, blk_lse, mass, bytes;
+  size_t pool_bytes, sel_bytes;
+};
+
+HostSlot host_slot(long long c, long long N, long long D, long long block, size_t elem) {
+  const long long nB = (N + block - 1) / block, rows = c * nB;
+  auto take = [](size_t& off, size_t n) {
+    const size_t at = off;
+    off += (n + 255) & ~(size_t)255;
+    return at;
+  };
+  HostSlot s{};
+  size_t off = 0;
+  s.q = take(off, (size_t)(c * N * D) * elem);
+  s.k = take(off, (size_t)(c * N * D) * elem);
+  s.v = take(off, (size_t)(c * N * D) * elem);
+  s.out = take(off, (size_t)(c * N * D) * elem);
+  s.lse = take(off, (size_t)(c * N) * sizeof(float));
+  s.probs = take(off, (size_t)(rows * nB) * sizeof(float));
+  s.pool_bytes = pool_ws_bytes(c, nB, (int)D);
+  s.ws_pool = take(off, s.pool_bytes);
+  s.sel_bytes = select_ws_bytes(rows);
+  s.ws_sel = take(off, s.sel_bytes);
+  s.row_ptr = take(off, (size_t)(rows + 1) * sizeof(int32_t));
+  s.col_idx = take(off, (size_t)(rows * nB) * sizeof(int32_t));
+  s.blk_lse = take(off, (size_t)(rows * nB * block) * sizeof(float));
+  s.mass = take(off, (size_t)(rows * nB) * sizeof(float));
+  s.bytes = off;
+  return s;
+}
+
+int host_chunk(long long BH, int chunk_heads) {
+  long long c = chunk_heads > 0 ? chunk_heads : BH / 8;
+  if (c < 1) c = 1;
+  if (c > BH) c = BH;
+  return (int)c;
+}
+
+// The three streams and the events of the host-buffer pipeline, per device,
+// created on first use.  One call at a time enqueues on them (the mutex), so
+// a wait always refers to the event record of its own call.
+struct HostStreams {
+  bool init = false;
+  cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+  std::vector<cudaEvent_t> ev;
+  std::mutex mu;
+};
+HostStreams g_host[kMaxDevices];
+
+cudaError_t host_events(HostStreams& h, size_t n) {
+  while (h.ev.size() < n) {
+    cudaEvent_t e;
+    cudaError_t r = cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+    if (r != cudaSuccess) return r;
+    h.ev.push_back(e);
+  }
+  return cudaSuccess;
+}
 // fine means (2 * BH * nBf * D floats) and the fine row softmax (BH * nBf^2 floats)
 size_t hier_ws_bytes(long long BH, long long nBf, int D) {
   return (size_t)(2 * BH * nBf * D + BH * nBf * nBf) * sizeof(float);
@@ -415,6 +479,108 @@ dsa_status dsa_permute_tokens(const void* src, void* dst, dsa_dtype dt, int B, i
                                              inverse != 0, dev->err_word,
                                              static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "permute_tokens launch");
+  return DSA_OK;
+}
+
+size_t dsa_host_pipeline_workspace_size(dsa_dtype dt, int B, int H, int N, int D, int block,
+                                        int chunk_heads) {
+  if (dt != DSA_BF16 && dt != DSA_F32) return 0;
+  if (check_shape(B, H, N, D, block) != DSA_OK) return 0;
+  const int c = host_chunk((long long)B * H, chunk_heads);
+  return 2 * host_slot(c, N, D, block, dt == DSA_BF16 ? 2 : 4).bytes;
+}
+
+dsa_status dsa_sparse_attention_host(const void* q, const void* k, const void* v, dsa_dtype dt,
+                                     int B, int H, int N, int D, int block, float scale, float p,
+                                     int chunk_heads, void* out, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (dt != DSA_BF16 && dt != DSA_F32) return fail(DSA_ERR_INVALID_ARG, "dt must be DSA_BF16 or DSA_F32");
+  dsa_status st = check_shape(B, H, N, D, block);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !out || !workspace) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (!(p > 0.f && p <= 1.f)) return fail(DSA_ERR_INVALID_ARG, "p must be in (0, 1] (got %g)", (double)p);
+  if (!aligned(workspace, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const long long BH = (long long)B * H;
+  const int c = host_chunk(BH, chunk_heads);
+  const size_t elem = dt == DSA_BF16 ? 2 : 4;
+  const HostSlot L = host_slot(c, N, D, block, elem);
+  if (ws_bytes < 2 * L.bytes)
+    return fail(DSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, 2 * L.bytes);
+  const long long nB = (N + (long long)block - 1) / block;
+  if ((st = check_blocks_limit(c * nB, (int)nB)) != DSA_OK) return st;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  int id = 0;
+  cudaError_t e = cudaGetDevice(&id);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  HostStreams& h = g_host[id];
+  std::lock_guard<std::mutex> lock(h.mu);
+  if (!h.init) {
+    e = cudaStreamCreateWithFlags(&h.s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h.s_comp, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h.s_out, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
+    h.init = true;
+  }
+  const long long n_chunks = (BH + c - 1) / c;
+  // events: [0] start, [1] end, then in / comp / out done per chunk
+  if ((e = host_events(h, (size_t)(2 + 3 * n_chunks))) != cudaSuccess)
+    return cuda_fail(e, "cudaEventCreateWithFlags");
+  cudaEvent_t* ev = h.ev.data();
+  auto in_done = [&](long long i) { return ev[2 + 3 * i]; };
+  auto comp_done = [&](long long i) { return ev[3 + 3 * i]; };
+  auto out_done = [&](long long i) { return ev[4 + 3 * i]; };
+  cudaStream_t caller = static_cast<cudaStream_t>(stream);
+  auto ok = [&](cudaError_t r) { return (e = r) == cudaSuccess; };
+  if (!ok(cudaEventRecord(ev[0], caller)) || !ok(cudaStreamWaitEvent(h.s_in, ev[0], 0)))
+    return cuda_fail(e, "host pipeline start");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t head_bytes = (size_t)N * D * elem;
+  for (long long ci = 0; ci < n_chunks; ++ci) {
+    const long long h0 = ci * c, n = (h0 + c <= BH ? c : BH - h0);
+    uint8_t* slot = ws + (size_t)(ci & 1) * L.bytes;
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)n * head_bytes;
+    // copy-in: the slot's inputs are free once chunk ci - 2 has computed
+    if (ci >= 2 && !ok(cudaStreamWaitEvent(h.s_in, comp_done(ci - 2), 0))) break;
+    if (!ok(cudaMemcpyAsync(slot + L.q, static_cast<const uint8_t*>(q) + off, bytes,
+                            cudaMemcpyHostToDevice, h.s_in)) ||
+        !ok(cudaMemcpyAsync(slot + L.k, static_cast<const uint8_t*>(k) + off, bytes,
+                            cudaMemcpyHostToDevice, h.s_in)) ||
+        !ok(cudaMemcpyAsync(slot + L.v, static_cast<const uint8_t*>(v) + off, bytes,
+                            cudaMemcpyHostToDevice, h.s_in)) ||
+        !ok(cudaEventRecord(in_done(ci), h.s_in)))
+      break;
+    // compute: after the copy-in, and once the slot's O of chunk ci - 2 is out
+    if (!ok(cudaStreamWaitEvent(h.s_comp, in_done(ci), 0))) break;
+    if (ci >= 2 && !ok(cudaStreamWaitEvent(h.s_comp, out_done(ci - 2), 0))) break;
+    const int hn = (int)n;
+    const int rows = (int)(n * nB);
+    float* probs = reinterpret_cast<float*>(slot + L.probs);
+    int32_t* rp = reinterpret_cast<int32_t*>(slot + L.row_ptr);
+    int32_t* ci_idx = reinterpret_cast<int32_t*>(slot + L.col_idx);
+    float* lse = reinterpret_cast<float*>(slot + L.lse);
+    float* bl = reinterpret_cast<float*>(slot + L.blk_lse);
+    if ((st = dsa_pool_score(slot + L.q, slot + L.k, dt, 1, hn, N, D, block, scale, nullptr,
+                             nullptr, probs, slot + L.ws_pool, L.pool_bytes, h.s_comp)) != DSA_OK ||
+        (st = dsa_select_topp(probs, rows, (int)nB, p, nullptr, nullptr, rp, ci_idx,
+                              slot + L.ws_sel, L.sel_bytes, h.s_comp)) != DSA_OK ||
+        (st = dsa_attn_fwd(slot + L.q, slot + L.k, slot + L.v, dt, 1, hn, N, D, block, scale, rp,
+                           ci_idx, slot + L.out, lse, bl, h.s_comp)) != DSA_OK ||
+        (st = dsa_block_mass(lse, bl, 1, hn, N, block, rp, reinterpret_cast<float*>(slot + L.mass),
+                             h.s_comp)) != DSA_OK)
+      return st;  // the inner call set the message
+    if (!ok(cudaEventRecord(comp_done(ci), h.s_comp))) break;
+    // copy-out
+    if (!ok(cudaStreamWaitEvent(h.s_out, comp_done(ci), 0)) ||
+        !ok(cudaMemcpyAsync(static_cast<uint8_t*>(out) + off, slot + L.out, bytes,
+                            cudaMemcpyDeviceToHost, h.s_out)) ||
+        !ok(cudaEventRecord(out_done(ci), h.s_out)))
+      break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline enqueue");
+  if (!ok(cudaEventRecord(ev[1], h.s_out)) || !ok(cudaStreamWaitEvent(caller, ev[1], 0)))
+    return cuda_fail(e, "host pipeline end");
   return DSA_OK;
 }
 

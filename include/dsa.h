@@ -16,6 +16,8 @@
  *   dsa_attn_bwd     gradients of the attention for a fixed mask.
  *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
  *                    exact attention weights (the next mask of a schedule).
+ *   dsa_sparse_attention_host  the four calls above on host-resident Q, K, V
+ *                    (chunks of heads, copies overlapped with compute).
  *   dsa_selftest_wait_timeout, dsa_selftest_exp2_poly  self-tests.
  *   dsa_hilbert_order, dsa_gilbert_order, dsa_permute_tokens  token
  *                    reordering along a 3-D Hilbert curve (the enclosing
@@ -245,6 +247,45 @@ dsa_status dsa_attn_bwd(const void* q, const void* k, const void* v, const void*
 dsa_status dsa_block_mass(const float* lse, const float* blk_lse,
                           int B, int H, int N, int block, const int32_t* row_ptr,
                           float* mass, void* stream);
+
+/*
+ * The whole pipeline (dsa_pool_score, dsa_select_topp, dsa_attn_fwd,
+ * dsa_block_mass over all blocks, Top-p threshold p) on HOST-resident Q, K,
+ * V, with O written back to host memory.  Every (b, h) is an independent
+ * problem (DSV abstract: each head is its own work item), so the B*H axis is
+ * cut into chunks of `chunk_heads` heads that run on three streams the
+ * library keeps per device: the copy-in of chunk c+1 (host -> device) and
+ * the copy-out of chunk c-1 overlap the compute of chunk c.  Two device
+ * slots in `workspace` alternate; events keep a slot from being refilled
+ * before its compute, or its O before its copy-out, has finished.
+ *
+ *   q, k, v     host, [B, H, N, D] in dt, contiguous; page-locked (pinned)
+ *               for the copies to overlap (pageable memory works, with
+ *               copies that do not overlap).
+ *   out         host, [B, H, N, D] in dt, same rules.
+ *   p, scale    as in dsa_select_topp and dsa_pool_score / dsa_attn_fwd.
+ *   chunk_heads heads per chunk, 1 .. B*H; <= 0 picks max(1, B*H / 8).
+ *   workspace   device, >= dsa_host_pipeline_workspace_size(...) bytes with
+ *               the same shape and chunk_heads, 256-byte aligned.
+ * Asynchronous: the copy-in waits for the work already on `stream`, and
+ * `stream` waits for the last copy-out, so synchronising `stream` (or the
+ * device) makes O visible in `out`.  Calls on one device are serialised on
+ * its three pipeline streams.  Errors: those of the four calls (shape,
+ * limits), DSA_ERR_INVALID_ARG for null pointers, a small or misaligned
+ * workspace or p outside (0, 1]; device-side flags as for the four calls
+ * (dsa_device_status).
+ */
+dsa_status dsa_sparse_attention_host(const void* q, const void* k, const void* v, dsa_dtype dt,
+                                     int B, int H, int N, int D, int block, float scale, float p,
+                                     int chunk_heads, void* out, void* workspace,
+                                     size_t ws_bytes, void* stream);
+
+/* Device workspace bytes for dsa_sparse_attention_host (two slots of one
+ * chunk's device buffers: Q, K, V, O, lse, P, the CSR at full capacity,
+ * per-block log-sums and masses, and the score and selection workspaces);
+ * 0 for an invalid shape. */
+size_t dsa_host_pipeline_workspace_size(dsa_dtype dt, int B, int H, int N, int D, int block,
+                                        int chunk_heads);
 
 /*
  * Dense probability rows from the exact block masses of a CSR mask, so that

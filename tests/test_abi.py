@@ -180,3 +180,20 @@ def test_python_wrapper_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         _lib.lib()
+
+
+def test_host_pipeline_workspace_size_needs_no_gpu(lib):
+    L = lib
+    # bf16, 2 x 40 heads x 75,600 tokens x 128, block 128, 5 heads per chunk
+    a = L.dsa_host_pipeline_workspace_size(1, 2, 40, 75600, 128, 128, 5)
+    b = L.dsa_host_pipeline_workspace_size(1, 2, 40, 75600, 128, 128, 10)
+    assert 0 < a < b
+    # two slots of 5 heads hold at least Q, K, V and O in bf16
+    assert a >= 2 * 4 * 5 * 75600 * 128 * 2
+    # fp32 needs more than bf16; chunk <= 0 picks B*H / 8 heads
+    assert L.dsa_host_pipeline_workspace_size(0, 2, 40, 75600, 128, 128, 5) > a
+    assert L.dsa_host_pipeline_workspace_size(1, 2, 40, 75600, 128, 128, 0) == \
+        L.dsa_host_pipeline_workspace_size(1, 2, 40, 75600, 128, 128, 10)
+    # invalid dtype or head dimension
+    assert L.dsa_host_pipeline_workspace_size(7, 1, 1, 1000, 128, 128, 1) == 0
+    assert L.dsa_host_pipeline_workspace_size(1, 1, 1, 1000, 96, 128, 1) == 0
