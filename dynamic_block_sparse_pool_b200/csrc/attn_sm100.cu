@@ -21,16 +21,19 @@
 //              two quad shuffles; no warp waits for another
 //   warp  8    MMA issuer (one thread) and TMEM allocation (whole warp)
 //   warp  9    TMA loader of Q and K (one thread)
-//   warp 10    TMA loader of V and TMA store of O (one thread): the softmax
-//              warps leave a row's O in the V slot of the row's last block,
-//              which no MMA reads once that block's PV is done, and this
-//              thread stores it before the slot takes its next V tile
+//   warp 10    TMA loader of V and TMA store of O (one thread)
 //   warp 11    row scheduler: draws the next row, checks its column indices
 //              and marks its ragged key block while the current row runs
+//   warps 8-11 also write each row's O out, one tensor-memory lane quarter
+//              (32 rows) each: O / l as bf16 into the V slot of the row's
+//              last block (no MMA reads it once that block's PV is done),
+//              which warp 10 stores with TMA before the slot takes its next
+//              V tile.  The softmax warps only leave 1/l in shared memory
+//              and go on to the next row.
 // Tensor memory (512 columns): three S buffers at columns 0, 128, 256 and O
 // at column 384.  Shared memory: Q, a 3-deep K ring and a 3-deep V ring of
 // [128 x D] tiles (a V slot doubles as the staging tile of a row's O), two
-// row-descriptor slots.
+// row-descriptor slots, 1/l of two rows.
 //
 // Blocks are numbered g = 0, 1, 2, ... across all the rows a CTA takes, in
 // order; block g uses K/V ring stage g % 3 and S buffer g % 3, so the rings
@@ -39,11 +42,20 @@
 // softmax.  Within a row the MMA thread issues S(0), S(1), S(2), then for
 // every block PV(it) [after P(it) is ready], S(it+3); the next row's S(0..2)
 // follow its last PV.  tcgen05 MMAs from one thread execute in order, so
-// S(g+3) overwrites buffer g % 3 only after PV(g) has read P(g) from it, and
-// a row's first PV (which overwrites O) runs only after every softmax warp
-// has read the previous row's O (each warp reads it before it writes its
-// first P of the next row).  Q of a row loads once every S of the previous
-// rows is done.
+// S(g+3) overwrites buffer g % 3 only after PV(g) has read P(g) from it.  A
+// row's first PV overwrites O, so the MMA warp issues it only once warps
+// 8-11 have read the previous row's O (OFree); each of them does so at a
+// point where it waits for nothing that the next row's PVs produce (the MMA
+// warp after the next row's first S products, the Q/K loader after its first
+// K tiles, the scheduler once the softmax warps are done with the row, the V
+// loader before it refills the staging slot or waits for a descriptor two
+// rows on).  The softmax warps can finish the next row before that (a row of
+// at most three blocks needs no PV of its own), so 1/l and its LReady
+// barrier alternate by row parity; they cannot get two rows ahead, because
+// the MMA warp issues the S products of the row after next only after that
+// OFree wait.  Q of a row loads once every S of the previous rows is done.
+// (A CPU model of this protocol, with random timing, checks that no wait
+// skips a phase, nothing deadlocks and no buffer is overwritten early.)
 //
 // Online softmax with a lazy reference: the first block's row maxima set the
 // reference m_ref; later blocks form P = 2^(S*scale*log2e - m_ref) without
@@ -82,6 +94,8 @@ constexpr int kSBufs = 3;       // S/P buffers in tensor memory
 constexpr int kRowSlots = 2;    // row descriptors in flight (current, next)
 // warps that read a row descriptor: 8 softmax, the MMA issuer, two loaders
 constexpr int kRowUsers = kSoftmaxThreads / 32 + 3;
+// warps 8-11 also write O out: their tensor-memory lane quarters are 0-3
+constexpr int kEpilogueWarps = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 384;
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -104,7 +118,9 @@ enum : int {
   kBarRowFull = kBarPVDone + kStages,   // + slot: row descriptor written
   kBarRowFree = kBarRowFull + kRowSlots,  // + slot: every user is done with it
   kBarOStaged = kBarRowFree + kRowSlots,  // + (row % 3): the row's O is in shared memory
-  kBarDrain = kBarOStaged + kStages,    // teardown after an abort: every MMA issued is done
+  kBarLReady = kBarOStaged + kStages,   // + (row % 2): the row's 1/l is in shared memory (8 softmax warps)
+  kBarOFree = kBarLReady + 2,           // the row's O is read out of tensor memory (4 warps)
+  kBarDrain = kBarOFree + 1,            // teardown after an abort: every MMA issued is done
   kNumBars = kBarDrain + 1
 };
 
@@ -127,7 +143,8 @@ struct SmemLayout {
   static constexpr int kV = kK + kStages * kTile;         // V ring
   static constexpr int kBar = kV + kStages * kTile;
   static constexpr int kRow = kBar + 8 * kNumBars;        // RowDesc [kRowSlots]
-  static constexpr int kSlot = kRow + kRowSlots * (int)sizeof(RowDesc);  // TMEM base, abort flag
+  static constexpr int kInvL = kRow + kRowSlots * (int)sizeof(RowDesc);  // float [2][128]: 1/l by row parity
+  static constexpr int kSlot = kInvL + 2 * BM * 4;                      // TMEM base, abort flag
   static constexpr int kBytes = kSlot + 16;
 };
 
@@ -177,35 +194,6 @@ constexpr int poly_chunks() { return D == 64 ? DSA_POLY_CHUNKS_D64 : DSA_POLY_CH
 // chunk k of 16 takes the polynomial path: the kPoly chunks are spread evenly
 __host__ __device__ constexpr bool poly_chunk(int k, int kPoly) {
   return (k + 1) * kPoly / 16 != k * kPoly / 16;
-}
-
-// 4 x 4 transpose of 32-bit words across the four threads of a quad (lanes
-// 4q .. 4q+3, t = lane % 4): afterwards x[u] holds what thread u held in
-// x[t].  Two butterfly steps: transpose the 2 x 2 blocks (partner t ^ 1),
-// then swap the off-diagonal blocks (partner t ^ 2).
-__device__ __forceinline__ void quad_transpose(uint32_t (&x)[4], int t) {
-  const bool odd = (t & 1) != 0, high = (t & 2) != 0;
-  uint32_t s0 = odd ? x[0] : x[1], s1 = odd ? x[2] : x[3];
-  s0 = __shfl_xor_sync(0xffffffffu, s0, 1);
-  s1 = __shfl_xor_sync(0xffffffffu, s1, 1);
-  if (odd) {
-    x[0] = s0;
-    x[2] = s1;
-  } else {
-    x[1] = s0;
-    x[3] = s1;
-  }
-  s0 = high ? x[0] : x[2];
-  s1 = high ? x[1] : x[3];
-  s0 = __shfl_xor_sync(0xffffffffu, s0, 2);
-  s1 = __shfl_xor_sync(0xffffffffu, s1, 2);
-  if (high) {
-    x[0] = s0;
-    x[1] = s1;
-  } else {
-    x[2] = s0;
-    x[3] = s1;
-  }
 }
 
 template <int D>
@@ -261,7 +249,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         uint32_t count = 1;
         if (i >= kBarPFull && i < kBarPFull + kStages) count = kSoftmaxThreads / 32;
         if (i >= kBarRowFree && i < kBarRowFree + kRowSlots) count = kRowUsers;
-        if (i >= kBarOStaged && i < kBarOStaged + kStages) count = kSoftmaxThreads / 32;
+        if (i >= kBarOStaged && i < kBarOStaged + kStages) count = kEpilogueWarps;
+        if (i == kBarLReady || i == kBarLReady + 1) count = kSoftmaxThreads / 32;
+        if (i == kBarOFree) count = kEpilogueWarps;
         mbar_init(bar(i), count);
       }
       *abort_flag = 0;
@@ -290,6 +280,54 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   auto row_wait = [&](int k) {
     return mbar_wait_idle(bar(kBarRowFull + (k & 1)), (uint32_t)(k >> 1) & 1u, kIdleSleepNs);
   };
+  // The O epilogue of one row, shared by warps 8-11 (each takes the 32 rows
+  // of its tensor-memory lane quarter, one row per thread, so the softmax
+  // warps go on to the next row at once): O / l as bf16 into the V slot of
+  // the row's last block gl (its PV is done, so no MMA reads that slot any
+  // more), in the O tensor map's 128-byte-swizzled layout (16-byte chunk k
+  // of row r of each 64-column sub-tile at chunk k ^ (r % 8)).  Then the
+  // warp arrives on OFree (it has read O: the next row's first PV may
+  // overwrite it) and on the row's OStaged (the V loader stores the tile).
+  // orow counts the rows with blocks; 1/l comes from the softmax warps
+  // (LReady).
+  float* inv_l = reinterpret_cast<float*>(smem + L::kInvL);
+  auto o_epilogue = [&](uint32_t orow, uint32_t gl) -> bool {
+    if (!warp_all(mbar_wait(bar(kBarLReady + (orow & 1u)), (orow >> 1) & 1u))) return false;
+    const int row = 32 * (warp & 3) + lane;
+    const float inv = inv_l[(orow & 1u) * BM + row];
+    if (!warp_all(mbar_wait(bar(kBarPVDone + gl % kStages), (gl / kStages) & 1u))) return false;
+    tc_fence_after();
+    uint8_t* stage = smem + L::kV + (gl % kStages) * kTileBytes + row * 128;
+    const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kTmemO;
+#pragma unroll
+    for (int c32 = 0; c32 < D / 32; ++c32) {
+      uint32_t o[32];  // columns 32 c32 .. 32 c32 + 31 of the thread's row
+      tmem_ld32(taddr + 32 * c32, o);
+      tmem_wait_ld_regs(o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int ch = 4 * c32 + j;  // 8-column chunk of the row
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(o[8 * j + 2 * u]) * inv,
+                                                          __uint_as_float(o[8 * j + 2 * u + 1]) * inv);
+          w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(stage + (ch >> 3) * L::kSub + (((ch & 7) ^ (row & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    fence_proxy_async_smem();  // visible to the TMA store
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(bar(kBarOFree));
+      mbar_arrive(bar(kBarOStaged + orow % kStages));
+    }
+    return true;
+  };
+
   // Blocks issued by the loaders (for the teardown after an abort).
   uint32_t k_issued = 0, v_issued = 0, q_issued = 0;
   bool had_rows = false;  // the MMA issuer issued at least one MMA
@@ -297,13 +335,22 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp == kSchedWarp) {
     // -------------------------------------------------------------- scheduler
     bool ok = true;
-    for (int k = 0;; ++k) {
+    uint32_t g = 0, orow = 0;  // blocks and rows with blocks published so far
+    // the epilogue share this warp still owes for the row in each slot
+    bool owe0 = false, owe1 = false;
+    uint32_t orow0 = 0, orow1 = 0, gl0 = 0, gl1 = 0;
+    int k = 0;
+    for (;; ++k) {
       const int slot = k & 1;
       // slot is free once row k - 2's readers are done with it
       // (a row lasts microseconds: poll every quarter microsecond)
       if (k >= kRowSlots)
         ok = warp_all(mbar_wait_idle(bar(kBarRowFree + slot), (uint32_t)((k - kRowSlots) >> 1) & 1u,
                                      256u));
+      // the softmax warps are done with row k - 2: write out its O (this
+      // warp's quarter)
+      if (ok && (slot ? owe1 : owe0)) ok = o_epilogue(slot ? orow1 : orow0, slot ? gl1 : gl0);
+      if (slot) owe1 = false; else owe0 = false;
       if (*abort_flag) ok = false;
       int r = 0;
       if (lane == 0) r = ok ? (int)atomicAdd(&tickets[0], 1u) : rows;
@@ -329,121 +376,181 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
       }
       bad = __any_sync(0xffffffffu, bad);
+      const int n = bad ? 0 : s1 - s0;
       if (lane == 0) {
         if (bad) flag_error(err, kErrCsrIndex | kErrRowPtr);
         d->r = r;
         d->s0 = bad ? 0 : s0;
-        d->n = bad ? 0 : s1 - s0;
+        d->n = n;
         mbar_arrive(bar(kBarRowFull + slot));  // release: the descriptor is visible to the readers
       }
+      if (n > 0) {
+        if (slot) {
+          owe1 = true;
+          orow1 = orow;
+          gl1 = g + n - 1;
+        } else {
+          owe0 = true;
+          orow0 = orow;
+          gl0 = g + n - 1;
+        }
+        ++orow;
+        g += n;
+      }
     }
+    // the row before the end marker may still owe its share
+    if (ok && k >= 1 && (((k - 1) & 1) ? owe1 : owe0))
+      ok = o_epilogue(((k - 1) & 1) ? orow1 : orow0, ((k - 1) & 1) ? gl1 : gl0);
     if (!ok) {
       *abort_flag = 1;
       if (lane == 0) flag_error(err, kErrTimeout);
     }
   } else if (warp == kKLoadWarp) {
     // ------------------------------------------------------------ Q/K loader
-    if (lane == 0) {
-      bool ok = true;
-      uint32_t g = 0;  // blocks of the rows before this one
-      for (int k = 0; ok; ++k) {
-        ok = row_wait(k) && !*abort_flag;
+    // The whole warp runs the loop (it also writes out a quarter of each
+    // row's O); lane 0 issues the copies.
+    const bool leader = lane == 0;
+    bool ok = true;
+    uint32_t g = 0, orow = 0;  // blocks and rows with blocks so far
+    bool owe = false;          // the previous row's epilogue share
+    uint32_t owe_orow = 0, owe_gl = 0;
+    for (int k = 0; ok; ++k) {
+      ok = warp_all(row_wait(k) && !*abort_flag);
+      if (!ok) break;
+      const RowDesc* d = rdesc + (k & 1);
+      const int r = d->r, s0 = d->s0, n = d->n;
+      if (r < 0) break;
+      __syncwarp();
+      if (leader) mbar_arrive(bar(kBarRowFree + (k & 1)));
+      if (n == 0) continue;
+      const int bh = r / nB, q0 = (r - bh * nB) * BM;
+      // Q's buffer is free once every S of the earlier rows is done
+      if (g > 0) {
+        ok = warp_all(mbar_wait_idle(bar(kBarSFull + (g - 1) % kStages), ((g - 1) / kStages) & 1u,
+                                     kIdleSleepNs) && !*abort_flag);
         if (!ok) break;
-        const RowDesc* d = rdesc + (k & 1);
-        const int r = d->r, s0 = d->s0, n = d->n;
-        if (r < 0) break;
-        mbar_arrive(bar(kBarRowFree + (k & 1)));
-        if (n == 0) continue;
-        const int bh = r / nB, q0 = (r - bh * nB) * BM;
-        // Q's buffer is free once every S of the earlier rows is done
-        if (g > 0) {
-          ok = mbar_wait_idle(bar(kBarSFull + (g - 1) % kStages), ((g - 1) / kStages) & 1u, kIdleSleepNs) &&
-               !*abort_flag;
-          if (!ok) break;
-        }
+      }
+      if (leader) {
         mbar_expect_tx(bar(kBarQ), kTileBytes);
         tma_tile<D>(sQ, &tmQ, q0, bh, bar(kBarQ));
-        ++q_issued;
-        for (int it = 0; it < n; ++it, ++g) {
-          const uint32_t s = g % kStages;
+      }
+      ++q_issued;
+      for (int it = 0; it < n; ++it, ++g) {
+        const uint32_t s = g % kStages;
+        // K slot s is free once S(g - 3) is done
+        ok = warp_all(mbar_wait_idle(bar(kBarSFull + s), ((g / kStages) & 1u) ^ 1u, kIdleSleepNs) &&
+                      !*abort_flag);
+        if (!ok) break;
+        if (leader) {
           const int j = col_idx[s0 + it];
-          // K slot s is free once S(g - 3) is done
-          ok = mbar_wait_idle(bar(kBarSFull + s), ((g / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
-          if (!ok) break;
           mbar_expect_tx(bar(kBarKFull + s), kTileBytes);
           tma_tile<D>(sK + s * kTileBytes, &tmK, j * BN, bh, bar(kBarKFull + s));
-          k_issued = g + 1;
+        }
+        k_issued = g + 1;
+        // with this row's first K tiles on their way, write out the
+        // previous row's O (the next K tile waits for this row's S(0))
+        if (owe && (it == 2 || it == n - 1)) {
+          owe = false;
+          if (!(ok = o_epilogue(owe_orow, owe_gl))) break;
         }
       }
-      if (!ok) {
-        *abort_flag = 1;
-        flag_error(err, kErrTimeout);
-      }
+      if (!ok) break;
+      owe = true;
+      owe_orow = orow++;
+      owe_gl = g - 1;
+    }
+    if (ok && owe) ok = o_epilogue(owe_orow, owe_gl);
+    if (!ok) {
+      *abort_flag = 1;
+      if (leader) flag_error(err, kErrTimeout);
     }
   } else if (warp == kVLoadWarp) {
     // -------------------------------------------------------------- V loader
-    // Also stores O: the softmax warps leave a row's O (bf16, in the tensor
-    // map's 128-byte-swizzled layout) in the V slot of the row's last block,
-    // which no MMA reads any more, and this thread stores it with TMA before
-    // it loads the next V tile into that slot (or at the end).
-    if (lane == 0) {
-      bool ok = true;
-      uint32_t g = 0;      // blocks of the rows so far
-      uint32_t orows = 0;  // rows with blocks so far
-      // rows whose O waits in a V slot, oldest first: at most three (their
-      // last blocks are among the three blocks before the next V load)
-      struct Pending {
-        uint32_t last, idx;  // the row's last block; its number among rows with blocks
-        int bh, q0;
-      };
-      Pending p0{}, p1{}, p2{};
-      int np = 0;
-      auto store_o = [&]() -> bool {  // the oldest pending row
-        if (!mbar_wait(bar(kBarOStaged + p0.idx % kStages), (p0.idx / kStages) & 1u)) return false;
+    // Also stores O: warps 8-11 leave a row's O (bf16, in the tensor map's
+    // 128-byte-swizzled layout) in the V slot of the row's last block, which
+    // no MMA reads any more, and this warp stores it with TMA before it loads
+    // the next V tile into that slot (or at the end).  The whole warp runs
+    // the loop (it writes out a quarter of each row's O); lane 0 issues the
+    // copies.
+    const bool leader = lane == 0;
+    bool ok = true;
+    uint32_t g = 0;      // blocks of the rows so far
+    uint32_t orows = 0;  // rows with blocks so far
+    // rows whose O is not stored yet, oldest first: at most three (their
+    // last blocks are among the three blocks before the next V load)
+    struct Pending {
+      uint32_t last, idx;  // the row's last block; its number among rows with blocks
+      int bh, q0, k;       // where its O goes; its descriptor number
+      bool shared;         // this warp's quarter of its O is staged
+    };
+    Pending p0{}, p1{}, p2{};
+    int np = 0;
+    auto share = [&](Pending& p) -> bool {
+      if (p.shared) return true;
+      p.shared = true;
+      return o_epilogue(p.idx, p.last);
+    };
+    auto store_o = [&]() -> bool {  // the oldest pending row
+      if (!share(p0)) return false;
+      if (!warp_all(mbar_wait(bar(kBarOStaged + p0.idx % kStages), (p0.idx / kStages) & 1u)))
+        return false;
+      if (leader) {
         const uint32_t src = sV + (p0.last % kStages) * kTileBytes;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, src + c * L::kSub, c * 64, p0.q0, p0.bh);
         tma_store_commit();
         tma_store_wait_read();  // the slot may be refilled now
-        p0 = p1;
-        p1 = p2;
-        --np;
-        return true;
-      };
-      for (int k = 0; ok; ++k) {
-        ok = row_wait(k) && !*abort_flag;
+      }
+      __syncwarp();
+      p0 = p1;
+      p1 = p2;
+      --np;
+      return true;
+    };
+    for (int k = 0; ok; ++k) {
+      // A row's share of O is written before this warp waits for the
+      // descriptor two rows on: that descriptor comes only once the softmax
+      // warps are done with the row between, whose first PV waits for the
+      // share (OFree).
+      if (np > 0 && p0.k <= k - 2 && !(ok = share(p0))) break;
+      if (np > 1 && p1.k <= k - 2 && !(ok = share(p1))) break;
+      if (np > 2 && p2.k <= k - 2 && !(ok = share(p2))) break;
+      ok = warp_all(row_wait(k) && !*abort_flag);
+      if (!ok) break;
+      const RowDesc* d = rdesc + (k & 1);
+      const int r = d->r, s0 = d->s0, n = d->n;
+      if (r < 0) break;
+      __syncwarp();
+      if (leader) mbar_arrive(bar(kBarRowFree + (k & 1)));
+      if (n == 0) continue;
+      const int bh = r / nB;
+      for (int it = 0; it < n; ++it, ++g) {
+        const uint32_t s = g % kStages;
+        // slot s last held V(g - 3); if that was a row's last block, the
+        // row's O is staged there
+        if (np > 0 && p0.last + kStages == g && !(ok = store_o())) break;
+        // V slot s is free once PV(g - 3) is done
+        ok = warp_all(mbar_wait_idle(bar(kBarPVDone + s), ((g / kStages) & 1u) ^ 1u, kIdleSleepNs) &&
+                      !*abort_flag);
         if (!ok) break;
-        const RowDesc* d = rdesc + (k & 1);
-        const int r = d->r, s0 = d->s0, n = d->n;
-        if (r < 0) break;
-        mbar_arrive(bar(kBarRowFree + (k & 1)));
-        if (n == 0) continue;
-        const int bh = r / nB;
-        for (int it = 0; it < n; ++it, ++g) {
-          const uint32_t s = g % kStages;
+        if (leader) {
           const int j = col_idx[s0 + it];
-          // slot s last held V(g - 3); if that was a row's last block, the
-          // row's O is staged there
-          if (np > 0 && p0.last + kStages == g && !(ok = store_o())) break;
-          // V slot s is free once PV(g - 3) is done
-          ok = mbar_wait_idle(bar(kBarPVDone + s), ((g / kStages) & 1u) ^ 1u, kIdleSleepNs) && !*abort_flag;
-          if (!ok) break;
           mbar_expect_tx(bar(kBarVFull + s), kTileBytes);
           tma_tile<D>(sV + s * kTileBytes, &tmV, j * BN, bh, bar(kBarVFull + s));
-          v_issued = g + 1;
         }
-        if (!ok) break;
-        const Pending pr{g - 1, orows++, bh, (r - bh * nB) * BM};
-        if (np == 0) p0 = pr;
-        else if (np == 1) p1 = pr;
-        else p2 = pr;
-        ++np;
+        v_issued = g + 1;
       }
-      while (ok && np > 0) ok = store_o();
-      if (!ok) {
-        *abort_flag = 1;
-        flag_error(err, kErrTimeout);
-      }
+      if (!ok) break;
+      const Pending pr{g - 1, orows++, bh, (r - bh * nB) * BM, k, false};
+      if (np == 0) p0 = pr;
+      else if (np == 1) p1 = pr;
+      else p2 = pr;
+      ++np;
+    }
+    while (ok && np > 0) ok = store_o();
+    if (!ok) {
+      *abort_flag = 1;
+      if (leader) flag_error(err, kErrTimeout);
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issuer
@@ -505,6 +612,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     using S1 = std::integral_constant<int, 1>;
     using S2 = std::integral_constant<int, 2>;
     uint32_t g = 0, qrows = 0;
+    bool owe = false;  // the previous row's epilogue share
+    uint32_t owe_orow = 0, owe_gl = 0;
     for (int k = 0; ok; ++k) {
       ok = warp_all(row_wait(k));
       if (!ok) break;
@@ -525,6 +634,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           default: issue_s(gs, S2{}); break;
         }
       }
+      // With this row's first S products queued, write out the previous
+      // row's O (this warp's quarter); this row's first PV overwrites O, so
+      // it waits until all four quarters are read (OFree).
+      if (ok && owe) {
+        owe = false;
+        ok = o_epilogue(owe_orow, owe_gl) && warp_all(mbar_wait(bar(kBarOFree), owe_orow & 1u));
+      }
       for (int it = 0; it < n && ok; ++it) {
         const uint32_t gb = g + it;
         const bool more = it + kStages < n;
@@ -534,8 +650,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           default: block(gb, it == 0, more, S2{}); break;
         }
       }
+      owe = true;
+      owe_orow = qrows - 1;  // rows with blocks before this one
+      owe_gl = g + n - 1;
       g += n;
     }
+    if (ok && owe) ok = o_epilogue(owe_orow, owe_gl);
     if (!ok && leader) {
       *abort_flag = 1;
       flag_error(err, kErrTimeout);
@@ -548,7 +668,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t lane_off = (uint32_t)rbase << 16;
     bool failed = false;
     uint32_t g = 0;      // blocks of the rows so far
-    uint32_t orows = 0;  // rows with blocks so far (their O went through a V slot)
+    uint32_t orows = 0;  // rows with blocks so far
     for (int k = 0; !failed; ++k) {
       if (!warp_all(row_wait(k))) {
         failed = true;
@@ -731,62 +851,18 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
         l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-        // lse and 1/l need only the row sums: they are done while the last
-        // PV runs
-        if (t0 == 0 && lse != nullptr) {
-          if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
-          if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
-        }
-        const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
-        const uint32_t gl = g + n - 1;
-        if (!warp_all(mbar_wait(bar(kBarPVDone + gl % kStages), (gl / kStages) & 1u))) {
-          failed = true;
-          break;
-        }
-        tc_fence_after();
-        // O / l as bf16 into the V slot of the row's last block (PV of that
-        // block is done, so no MMA reads it any more), in the O tensor map's
-        // 128-byte-swizzled layout: 16-byte chunk k of row r of each 64-column
-        // sub-tile sits at chunk k ^ (r % 8).  The V loader stores the tile
-        // with TMA.  This warp's reads of O are done (tcgen05.wait::ld)
-        // before it writes the next row's first P, which is what lets that
-        // row's first PV overwrite O.  The four threads of a quad swap their
-        // packed pairs so that each holds 8 consecutive columns of one row
-        // and writes them as one 16-byte chunk.
-        uint32_t o[64];  // o[4k + u]: row ra, column 8k + 2*t0 + u; o[4k + 2 + u]: row rb
-        if constexpr (D == 128) {
-          tmem_ld16x256b_x16(tmem + lane_off + kTmemO, o);
-          tmem_wait_ld_regs64(o);
-        } else {
-          uint32_t(&o32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
-          tmem_ld16x256b_x8(tmem + lane_off + kTmemO, o32);
-          tmem_wait_ld_regs(o32);
-        }
-        uint8_t* stage = smem + L::kV + (gl % kStages) * kTileBytes;
-#pragma unroll
-        for (int h = 0; h < D / 32; ++h) {  // chunks 4h .. 4h+3 (columns 32h .. 32h+31)
-          uint32_t xa[4], xb[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int kc = 4 * h + j;
-            const __nv_bfloat162 ha = __floats2bfloat162_rn(__uint_as_float(o[4 * kc]) * inv_a,
-                                                            __uint_as_float(o[4 * kc + 1]) * inv_a);
-            const __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[4 * kc + 2]) * inv_b,
-                                                            __uint_as_float(o[4 * kc + 3]) * inv_b);
-            xa[j] = *reinterpret_cast<const uint32_t*>(&ha);
-            xb[j] = *reinterpret_cast<const uint32_t*>(&hb);
+        // lse, and 1/l for the warps that write O out (warps 8-11, once the
+        // last PV is done); this warp goes on to the next row at once
+        if (t0 == 0) {
+          if (lse != nullptr) {
+            if (ra < qlen) lse[(size_t)bh * N + q0 + ra] = (mref_a + log2f(l_a)) * kLn2;
+            if (rb < qlen) lse[(size_t)bh * N + q0 + rb] = (mref_b + log2f(l_b)) * kLn2;
           }
-          quad_transpose(xa, t0);  // xa[u]: columns 8(4h + t0) + 2u, +1
-          quad_transpose(xb, t0);
-          const int ch = 4 * h + t0, c = ch >> 3, kk = ch & 7;
-          *reinterpret_cast<uint4*>(stage + c * L::kSub + ra * 128 + ((kk ^ (ra & 7)) << 4)) =
-              make_uint4(xa[0], xa[1], xa[2], xa[3]);
-          *reinterpret_cast<uint4*>(stage + c * L::kSub + rb * 128 + ((kk ^ (rb & 7)) << 4)) =
-              make_uint4(xb[0], xb[1], xb[2], xb[3]);
+          inv_l[(orows & 1u) * BM + ra] = 1.0f / l_a;
+          inv_l[(orows & 1u) * BM + rb] = 1.0f / l_b;
         }
-        fence_proxy_async_smem();  // visible to the TMA store
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarOStaged + orows % kStages));
+        if (lane == 0) mbar_arrive(bar(kBarLReady + (orows & 1u)));  // release: 1/l is visible
         ++orows;
       } else {
         __nv_bfloat16* ra_out = out + ((size_t)bh * N + q0 + ra) * D;
