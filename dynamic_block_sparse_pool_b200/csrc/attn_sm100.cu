@@ -383,6 +383,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         d->s0 = bad ? 0 : s0;
         d->n = n;
         mbar_arrive(bar(kBarRowFull + slot));  // release: the descriptor is visible to the readers
+        // the row's Q tile into L2 now: its load then has the current row's
+        // time to come from HBM, and the MMA warp can start the row's first
+        // S products before the current row's last PV
+        if (n > 0) {
+          const int bh = r / nB, q0 = (r - bh * nB) * BM;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) tma_prefetch_l2_3d(&tmQ, c * 64, q0, bh);
+        }
       }
       if (n > 0) {
         if (slot) {
@@ -614,6 +622,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint32_t g = 0, qrows = 0;
     bool owe = false;  // the previous row's epilogue share
     uint32_t owe_orow = 0, owe_gl = 0;
+    int ahead = 0;     // S products of this row issued during the previous one
+    uint32_t orow = 0; // rows with blocks so far
+    auto issue_s_any = [&](uint32_t gs) {
+      switch (gs % kStages) {
+        case 0: issue_s(gs, S0{}); break;
+        case 1: issue_s(gs, S1{}); break;
+        default: issue_s(gs, S2{}); break;
+      }
+    };
     for (int k = 0; ok; ++k) {
       ok = warp_all(row_wait(k));
       if (!ok) break;
@@ -623,17 +640,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       __syncwarp();
       if (leader) mbar_arrive(bar(kBarRowFree + (k & 1)));
       if (n == 0) continue;
-      ok = warp_all(mbar_wait(bar(kBarQ), qrows & 1u));
-      ++qrows;
-      had_rows = true;
-      for (int it = 0; it < 3 && it < n && ok; ++it) {
-        const uint32_t gs = g + it;
-        switch (gs % kStages) {
-          case 0: issue_s(gs, S0{}); break;
-          case 1: issue_s(gs, S1{}); break;
-          default: issue_s(gs, S2{}); break;
-        }
+      const uint32_t this_orow = orow++;
+      if (ahead == 0) {
+        ok = warp_all(mbar_wait(bar(kBarQ), qrows & 1u));
+        ++qrows;
       }
+      had_rows = true;
+      for (int it = ahead; it < 3 && it < n && ok; ++it) issue_s_any(g + it);
+      ahead = 0;
       // With this row's first S products queued, write out the previous
       // row's O (this warp's quarter); this row's first PV overwrites O, so
       // it waits until all four quarters are read (OFree).
@@ -649,9 +663,27 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           case 1: block(gb, it == 0, more, S1{}); break;
           default: block(gb, it == 0, more, S2{}); break;
         }
+        // Before this row's last PV: if the next row is published and its Q
+        // has landed, issue its first two S products now (their buffers held
+        // P of this row's blocks n-3 and n-2, whose PVs are issued), so they
+        // are ready when the softmax warps finish this row.  Checks only: if
+        // either is not there yet they follow the last PV as usual.
+        if (it == n - 2 && ok) {
+          const int k1 = k + 1;
+          if (warp_all(mbar_try_wait(bar(kBarRowFull + (k1 & 1)), (uint32_t)(k1 >> 1) & 1u))) {
+            const RowDesc* d1 = rdesc + (k1 & 1);
+            const int r1 = d1->r, n1 = d1->n;
+            if (r1 >= 0 && n1 > 0 && warp_all(mbar_try_wait(bar(kBarQ), qrows & 1u))) {
+              ++qrows;
+              ahead = n1 >= 2 ? 2 : 1;
+              tc_fence_after();
+              for (int a = 0; a < ahead && ok; ++a) issue_s_any(g + n + a);
+            }
+          }
+        }
       }
       owe = true;
-      owe_orow = qrows - 1;  // rows with blocks before this one
+      owe_orow = this_orow;
       owe_gl = g + n - 1;
       g += n;
     }
