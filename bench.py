@@ -47,8 +47,8 @@ ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn
 # prefix of attn_sm100.cu at capture time (scaled to the full workload when
 # the capture ran a smaller case); stale entries are ignored.
 ATTN_TRAFFIC = {
-    # 8-head Wan2.1-like capture: 642.1 MB read + 500.2 MB written, x5 heads
-    "0b6b551a47819654": int((642087936 + 500244480) * 5),
+    # 8-head Wan2.1-like capture: 727.3 MB read + 501.9 MB written, x5 heads
+    "f2ee7f556515a321": int((727342848 + 501897472) * 5),
 }
 
 
