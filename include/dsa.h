@@ -38,8 +38,12 @@
  *    in DSA_BF16 or DSA_F32.  D is 64 or 128; block is 64 or 128.
  *  - Every pointer argument is a DEVICE pointer owned by the caller unless
  *    stated otherwise; the library keeps no reference after a call returns
- *    and allocates no device memory.  Scratch memory is passed in as
- *    `workspace` (size from dsa_workspace_size).
+ *    and allocates no device memory at call time.  Scratch memory is passed
+ *    in as `workspace` (size from dsa_workspace_size).  What the library
+ *    itself holds per device, for the life of the process: the device
+ *    error word and the attention's ticket counters (module data, 32 KB),
+ *    the static selection scratch of dsa_select_topp_static, and, once
+ *    dsa_sparse_attention_host has run, three streams and a pool of events.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and never synchronises the host, except
  *    dsa_device_status.
