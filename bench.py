@@ -44,11 +44,13 @@ METRIC = "block-sparse attn fwd TFLOP/s (executed) & % bf16 peak; speedup vs p=1
 LAUNCHES_PER_STEP = 7  # pool_means, block_scores, select, csr_scan, compact, attn_fwd, block_mass
 ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn_sm100.cu")
 # DRAM bytes per attention launch from an ncu capture, keyed by the sha256
-# prefix of attn_sm100.cu at capture time (scaled to the full workload when
-# the capture ran a smaller case); stale entries are ignored.
+# prefix of attn_sm100.cu at capture time: (workload, p, seed, heads of the
+# capture, bytes read + written).  Reported only for that workload, p and
+# seed, scaled by the number of heads (traffic grows with the heads); stale
+# entries are ignored.
 ATTN_TRAFFIC = {
-    # 8-head Wan2.1-like capture: 727.3 MB read + 501.9 MB written, x5 heads
-    "f2ee7f556515a321": int((727342848 + 501897472) * 5),
+    # 8-head Wan2.1-like capture: 727.3 MB read + 501.9 MB written
+    "f2ee7f556515a321": ("wan2.1-14b-like", 0.9, 0, 8, 727342848 + 501897472),
 }
 
 
@@ -648,7 +650,12 @@ def main():
         "config": config_of(w, args),
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
     }
-    traffic = ATTN_TRAFFIC.get(attn_source_hash())
+    traffic = None
+    entry = ATTN_TRAFFIC.get(attn_source_hash())
+    if entry is not None:
+        name, p_cap, seed_cap, heads_cap, nbytes = entry
+        if w.name == name and args.p == p_cap and args.seed == seed_cap and w.batch == 1:
+            traffic = int(nbytes * w.heads / heads_cap)
     # The denominator is the measured burst cuBLAS bf16 rate: the sustained
     # figure was taken at a lower median SM clock than this loop runs at, so
     # it would flatter the fraction; it is reported beside it for context.
