@@ -41,7 +41,8 @@ import torch  # noqa: E402
 from dynamic_block_sparse_pool_b200 import ops, synth  # noqa: E402
 
 METRIC = "block-sparse attn fwd TFLOP/s (executed) & % bf16 peak; speedup vs p=1"
-LAUNCHES_PER_STEP = 7  # pool_means, block_scores, select, csr_scan, compact, attn_fwd, block_mass
+# pool_means, block_scores, select, csr_scan, compact, row_order, attn_fwd, block_mass
+LAUNCHES_PER_STEP = 8
 ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn_sm100.cu")
 # DRAM bytes per attention launch from an ncu capture, keyed by the sha256
 # prefix of attn_sm100.cu at capture time: (workload, p, seed, heads of the
@@ -49,8 +50,8 @@ ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_pool_b200", "csrc", "attn
 # seed, scaled by the number of heads (traffic grows with the heads); stale
 # entries are ignored.
 ATTN_TRAFFIC = {
-    # 8-head Wan2.1-like capture: 727.3 MB read + 501.9 MB written
-    "f2ee7f556515a321": ("wan2.1-14b-like", 0.9, 0, 8, 727342848 + 501897472),
+    # 8-head Wan2.1-like capture: 539.2 MB read + 500.2 MB written
+    "2de04737e0c4a4a4": ("wan2.1-14b-like", 0.9, 0, 8, 539209728 + 500218880),
 }
 
 
@@ -328,6 +329,7 @@ def sweep(args):
         wsel = torch.empty(ops.workspace_size(1, B, H, N, D, blk), device=dev, dtype=torch.uint8)
         rp = torch.empty(rows + 1, device=dev, dtype=torch.int32)
         ci = torch.empty(rows * nB, device=dev, dtype=torch.int32)
+        order = torch.empty(rows, device=dev, dtype=torch.int32)
         out = torch.empty_like(q)
         lse = torch.empty(B, H, N, device=dev)
         cap = rows * nB if cand is None else int(cand[0][-1])
@@ -340,8 +342,10 @@ def sweep(args):
         else:
             score = lambda: ops.pool_score(q, k, blk, scale, cand=cand, out=P, workspace=wp)
         search = lambda: (score(),
-                          ops.select_topp(P, p, cand=cand, row_ptr=rp, col_idx=ci, workspace=wsel))
-        attend = lambda: ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=bl)
+                          ops.select_topp(P, p, cand=cand, row_ptr=rp, col_idx=ci, workspace=wsel),
+                          ops.row_order(rp, B, H, nB, out=order))
+        attend = lambda: ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=bl,
+                                      order=order)
         mass = lambda: ops.block_mass(lse, bl, rp, blk, mass=ms_)
         search(); attend(); mass(); ops.device_status(dev)
         flops, nnz = executed_flops(rp, ci, N, blk, D, nB)
@@ -597,14 +601,16 @@ def main():
     lse = torch.empty(B, H, N, device=dev, dtype=torch.float32)
     blk_lse = torch.empty(rows * nB, blk, device=dev, dtype=torch.float32)
     mass = torch.empty(rows * nB, device=dev, dtype=torch.float32)
+    order = torch.empty(rows, device=dev, dtype=torch.int32)
     stream = torch.cuda.current_stream(dev)
 
     def search():
         ops.pool_score(q, k, blk, scale, out=P, workspace=ws_pool)
         ops.select_topp(P, args.p, row_ptr=row_ptr, col_idx=col_idx, workspace=ws_sel)
+        ops.row_order(row_ptr, B, H, nB, out=order)
 
-    def attend(rp=row_ptr, ci=col_idx):
-        ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=blk_lse)
+    def attend(rp=row_ptr, ci=col_idx, ro=order):
+        ops.attn_fwd(q, k, v, rp, ci, blk, scale, out=out, lse=lse, blk_lse=blk_lse, order=ro)
 
     def finish(rp=row_ptr):
         ops.block_mass(lse, blk_lse, rp, blk, mass=mass)
@@ -684,7 +690,7 @@ def main():
     if not args.no_dense:
         rp_all = (torch.arange(rows + 1, device=dev, dtype=torch.int64) * nB).to(torch.int32)
         col_all = torch.arange(nB, device=dev, dtype=torch.int32).repeat(rows)
-        attend(rp_all, col_all)
+        attend(rp_all, col_all, None)  # equal rows: index order is the longest-first one
         torch.cuda.synchronize(dev)
 
         def back_to_back(fn, reps):
@@ -701,7 +707,7 @@ def main():
         k_dense = 4
         for _ in range(3):
             ms_sparse_alt = back_to_back(lambda: (search(), attend(), finish()), k_sparse)
-            ms_dense = back_to_back(lambda: attend(rp_all, col_all), k_dense)
+            ms_dense = back_to_back(lambda: attend(rp_all, col_all, None), k_dense)
         red = dense_flops / flops
         line["speedup_vs_p1"] = {
             "dense_attn_ms": ms_dense,

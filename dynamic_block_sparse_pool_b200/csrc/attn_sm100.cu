@@ -12,7 +12,10 @@
 // One CTA per SM.  Each CTA takes CSR rows (one query block of 128 rows
 // each) from a ticket counter shared by the launch until none are left, so
 // a CTA that drew short rows takes more of them (the balance of one CTA per
-// row, without a CTA's start-up and tear-down cost per row).  384 threads:
+// row, without a CTA's start-up and tear-down cost per row).  Ticket t is
+// row row_order[t] when an order is given: each head's rows longest first
+// put the short rows at the end of the launch, where they fill the gaps
+// the last long rows leave.  384 threads:
 //   warps 0-7  softmax: warp w owns the 16 query rows (TMEM lanes)
 //              32*(w%4) + 16*(w/4) .. +15; thread t of it owns two rows
 //              (t/4 and t/4 + 8 of those) and, in every 8-key chunk, keys
@@ -211,7 +214,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmO, int N, int nB, int rows,
                       float scale_log2, const int32_t* __restrict__ row_ptr,
-                      const int32_t* __restrict__ col_idx, __nv_bfloat16* __restrict__ out,
+                      const int32_t* __restrict__ col_idx,
+                      const int32_t* __restrict__ row_order, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ lse, float* __restrict__ blk_lse,
                       unsigned* __restrict__ tickets, unsigned* err) {
   using L = SmemLayout<D>;
@@ -352,8 +356,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (ok && (slot ? owe1 : owe0)) ok = o_epilogue(slot ? orow1 : orow0, slot ? gl1 : gl0);
       if (slot) owe1 = false; else owe0 = false;
       if (*abort_flag) ok = false;
-      int r = 0;
-      if (lane == 0) r = ok ? (int)atomicAdd(&tickets[0], 1u) : rows;
+      // ticket t is row row_order[t] (t itself without an order); an entry
+      // outside [0, rows) is reported and passed over for the next ticket
+      int r = rows;
+      if (lane == 0 && ok) {
+        for (;;) {
+          const unsigned t = atomicAdd(&tickets[0], 1u);
+          if (t >= (unsigned)rows) break;
+          const int o = row_order ? row_order[t] : (int)t;
+          if ((unsigned)o < (unsigned)rows) {
+            r = o;
+            break;
+          }
+          flag_error(err, kErrRowOrder);
+        }
+      }
       r = __shfl_sync(0xffffffffu, r, 0);
       RowDesc* d = rdesc + slot;
       if (r >= rows) {
@@ -990,7 +1007,7 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int D) {
 template <int D>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mo, int BH, int N, float scale, const int32_t* row_ptr, const int32_t* col_idx,
-                     void* out, float* lse, float* blk_lse, unsigned* tickets, int num_sms,
+                     const int32_t* row_order, void* out, float* lse, float* blk_lse, unsigned* tickets, int num_sms,
                      unsigned* err, cudaStream_t s) {
   const int nB = ceil_div(N, BN);
   const int rows = BH * nB;
@@ -1004,7 +1021,7 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   // file, so no second CTA fits beside one)
   const int grid = rows < num_sms ? rows : num_sms;
   attn_fwd_sm100_kernel<D><<<grid, kThreads, smem, s>>>(
-      mq, mk, mv, mo, N, nB, rows, scale_log2, row_ptr, col_idx, static_cast<__nv_bfloat16*>(out),
+      mq, mk, mv, mo, N, nB, rows, scale_log2, row_ptr, col_idx, row_order, static_cast<__nv_bfloat16*>(out),
       lse, blk_lse, tickets, err);
   return cudaGetLastError();
 }
@@ -1013,9 +1030,9 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int BH, int N,
                               int D, float scale, const int32_t* row_ptr,
-                              const int32_t* col_idx, void* out, float* lse, float* blk_lse,
-                              unsigned* tickets, int num_sms, unsigned* err, cudaStream_t s,
-                              const char** why) {
+                              const int32_t* col_idx, const int32_t* row_order, void* out,
+                              float* lse, float* blk_lse, unsigned* tickets, int num_sms,
+                              unsigned* err, cudaStream_t s, const char** why) {
   CUtensorMap mq, mk, mv, mo;
   if (!make_tile_map(&mq, q, BH, N, D) || !make_tile_map(&mk, k, BH, N, D) ||
       !make_tile_map(&mv, v, BH, N, D) || !make_tile_map(&mo, out, BH, N, D)) {
@@ -1023,10 +1040,10 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int B
     return cudaErrorInvalidValue;
   }
   if (D == 64)
-    return launch_d<64>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, tickets,
-                        num_sms, err, s);
-  return launch_d<128>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, out, lse, blk_lse, tickets,
-                       num_sms, err, s);
+    return launch_d<64>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, row_order, out, lse,
+                        blk_lse, tickets, num_sms, err, s);
+  return launch_d<128>(mq, mk, mv, mo, BH, N, scale, row_ptr, col_idx, row_order, out, lse,
+                       blk_lse, tickets, num_sms, err, s);
 }
 
 }  // namespace dsa

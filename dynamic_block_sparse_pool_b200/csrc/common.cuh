@@ -15,6 +15,7 @@ enum : unsigned {
   kErrTimeout = 8u,      // a bounded wait on an mbarrier ran out
   kErrAlign = 16u,       // dynamic shared memory not 1024-byte aligned
   kErrPerm = 32u,        // a token permutation entry outside [0, N)
+  kErrRowOrder = 64u,    // an attention row-order entry outside [0, rows)
 };
 
 // Upper bound for one mbarrier wait before a kernel gives up (nanoseconds).
@@ -52,11 +53,16 @@ cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, bool b
                              int BH, int N, int D, int block, float scale,
                              const int32_t* row_ptr, const int32_t* col_idx, void* out,
                              float* lse, float* blk_lse, unsigned* err, cudaStream_t s);
+// Each head's rows of a CSR mask by descending block count (ties by row
+// index), as global row indices: order[bh*nB .. (bh+1)*nB) holds head bh's.
+cudaError_t launch_row_order(const int32_t* row_ptr, int BH, int nB, int num_sms, int32_t* order,
+                             cudaStream_t s);
 // tickets: two zeroed words of device memory that no concurrent launch uses
-// (the kernel leaves them zeroed); num_sms: the device's SM count.
+// (the kernel leaves them zeroed); num_sms: the device's SM count; row_order:
+// the order in which the CTAs take the rows (NULL: index order).
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, int BH,
                               int N, int D, float scale, const int32_t* row_ptr,
-                              const int32_t* col_idx, void* out, float* lse,
+                              const int32_t* col_idx, const int32_t* row_order, void* out, float* lse,
                               float* blk_lse, unsigned* tickets, int num_sms,
                               unsigned* err, cudaStream_t s, const char** why);
 cudaError_t launch_mass_to_probs(const int32_t* row_ptr, const int32_t* col_idx,

@@ -129,7 +129,7 @@ size_t select_ws_bytes(long long rows) { return (size_t)(rows * 33) * sizeof(uin
 // Byte offsets of one chunk's device buffers inside a pipeline slot, each
 // 256-byte aligned; `bytes` is the slot's size.
 struct HostSlot {
-  size_t q, k, v, out, lse, probs, ws_pool, ws_sel, row_ptr, col_idx, blk_lse, mass, bytes;
+  size_t q, k, v, out, lse, probs, ws_pool, ws_sel, row_ptr, col_idx, order, blk_lse, mass, bytes;
   size_t pool_bytes, sel_bytes;
 };
 
@@ -154,6 +154,7 @@ HostSlot host_slot(long long c, long long N, long long D, long long block, size_
   s.ws_sel = take(off, s.sel_bytes);
   s.row_ptr = take(off, (size_t)(rows + 1) * sizeof(int32_t));
   s.col_idx = take(off, (size_t)(rows * nB) * sizeof(int32_t));
+  s.order = take(off, (size_t)rows * sizeof(int32_t));
   s.blk_lse = take(off, (size_t)(rows * nB * block) * sizeof(float));
   s.mass = take(off, (size_t)(rows * nB) * sizeof(float));
   s.bytes = off;
@@ -203,7 +204,7 @@ size_t bwd_ws_bytes(long long BH, long long nB, long long N) {
 
 extern "C" {
 
-int dsa_version(void) { return 100; }
+int dsa_version(void) { return 200; }
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
@@ -317,10 +318,27 @@ dsa_status dsa_select_topp(const float* probs, int rows, int nB, float p,
   return DSA_OK;
 }
 
+dsa_status dsa_row_order(const int32_t* row_ptr, int B, int H, int nB, int32_t* order,
+                         void* stream) {
+  g_last_error.clear();
+  if (!row_ptr || !order) return fail(DSA_ERR_INVALID_ARG, "null row_ptr or order");
+  if (B < 1 || H < 1) return fail(DSA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
+  if (nB < 1 || nB > DSA_MAX_BLOCKS) return fail(DSA_ERR_INVALID_ARG, "nB outside 1..DSA_MAX_BLOCKS");
+  if ((long long)B * H * nB >= INT_MAX) return fail(DSA_ERR_INVALID_ARG, "too many block rows");
+  if (!aligned(row_ptr, 4) || !aligned(order, 4)) return fail(DSA_ERR_INVALID_ARG, "misaligned pointer");
+  DeviceInfo* dev = nullptr;
+  dsa_status st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  cudaError_t e = dsa::launch_row_order(row_ptr, B * H, nB, dev->num_sms, order,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "row_order launch");
+  return DSA_OK;
+}
+
 dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype dt, int B, int H,
                         int N, int D, int block, float scale, const int32_t* row_ptr,
-                        const int32_t* col_idx, void* out, float* lse, float* blk_lse,
-                        void* stream) {
+                        const int32_t* col_idx, const int32_t* row_order, void* out, float* lse,
+                        float* blk_lse, void* stream) {
   g_last_error.clear();
   if (!q || !k || !v || !out || !row_ptr || !col_idx)
     return fail(DSA_ERR_INVALID_ARG, "null q, k, v, out, row_ptr or col_idx");
@@ -329,7 +347,8 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
   if (st != DSA_OK) return st;
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(lse, 4) || !aligned(blk_lse, 4))
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(row_order, 4) || !aligned(lse, 4) ||
+      !aligned(blk_lse, 4))
     return fail(DSA_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned; index and float arrays 4-byte aligned");
   DeviceInfo* dev = nullptr;
   if ((st = device_info(&dev)) != DSA_OK) return st;
@@ -339,8 +358,9 @@ dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype d
   if (dt == DSA_BF16 && block == 128 && N >= 128) {
     const char* why = nullptr;
     const unsigned pair = dev->next_pair.fetch_add(1u) % kTicketPairs;
-    e = dsa::launch_attn_sm100(q, k, v, BH, N, D, scale, row_ptr, col_idx, out, lse, blk_lse,
-                               dev->tickets + 2 * pair, dev->num_sms, dev->err_word, s, &why);
+    e = dsa::launch_attn_sm100(q, k, v, BH, N, D, scale, row_ptr, col_idx, row_order, out, lse,
+                               blk_lse, dev->tickets + 2 * pair, dev->num_sms, dev->err_word, s,
+                               &why);
     if (e != cudaSuccess && why) return fail(DSA_ERR_CUDA, "attn_fwd: %s", why);
   } else {
     e = dsa::launch_attn_simt(q, k, v, dt == DSA_BF16, BH, N, D, block, scale, row_ptr, col_idx,
@@ -559,14 +579,16 @@ dsa_status dsa_sparse_attention_host(const void* q, const void* k, const void* v
     float* probs = reinterpret_cast<float*>(slot + L.probs);
     int32_t* rp = reinterpret_cast<int32_t*>(slot + L.row_ptr);
     int32_t* ci_idx = reinterpret_cast<int32_t*>(slot + L.col_idx);
+    int32_t* order = reinterpret_cast<int32_t*>(slot + L.order);
     float* lse = reinterpret_cast<float*>(slot + L.lse);
     float* bl = reinterpret_cast<float*>(slot + L.blk_lse);
     if ((st = dsa_pool_score(slot + L.q, slot + L.k, dt, 1, hn, N, D, block, scale, nullptr,
                              nullptr, probs, slot + L.ws_pool, L.pool_bytes, h.s_comp)) != DSA_OK ||
         (st = dsa_select_topp(probs, rows, (int)nB, p, nullptr, nullptr, rp, ci_idx,
                               slot + L.ws_sel, L.sel_bytes, h.s_comp)) != DSA_OK ||
+        (st = dsa_row_order(rp, 1, hn, (int)nB, order, h.s_comp)) != DSA_OK ||
         (st = dsa_attn_fwd(slot + L.q, slot + L.k, slot + L.v, dt, 1, hn, N, D, block, scale, rp,
-                           ci_idx, slot + L.out, lse, bl, h.s_comp)) != DSA_OK ||
+                           ci_idx, order, slot + L.out, lse, bl, h.s_comp)) != DSA_OK ||
         (st = dsa_block_mass(lse, bl, 1, hn, N, block, rp, reinterpret_cast<float*>(slot + L.mass),
                              h.s_comp)) != DSA_OK)
       return st;  // the inner call set the message
@@ -625,13 +647,14 @@ dsa_status dsa_device_status(void* stream) {
   const unsigned zero = 0;
   e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
   if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
-  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s%s%s", word,
+  return fail(DSA_ERR_DEVICE, "device error word 0x%x:%s%s%s%s%s%s%s", word,
               (word & dsa::kErrCsrIndex) ? " csr-index-out-of-range" : "",
               (word & dsa::kErrRowPtr) ? " bad-row-ptr" : "",
               (word & dsa::kErrProb) ? " probability-outside-[0,1]" : "",
               (word & dsa::kErrTimeout) ? " wait-timeout" : "",
               (word & dsa::kErrAlign) ? " shared-memory-misaligned" : "",
-              (word & dsa::kErrPerm) ? " permutation-index-out-of-range" : "");
+              (word & dsa::kErrPerm) ? " permutation-index-out-of-range" : "",
+              (word & dsa::kErrRowOrder) ? " row-order-index-out-of-range" : "");
 }
 
 }  // extern "C"

@@ -19,9 +19,12 @@
 //   1024-bit mask (one ballot per register) plus a count.
 // Kernel 2 (scan): exclusive scan of the counts into row_ptr (one CTA).
 // Kernel 3 (compact): one warp per row writes the kept indices ascending.
+// Kernel 4 (row order, its own call): each head's rows by descending block
+//   count, the order in which the persistent attention kernel takes them.
 #include <cstring>
 
 #include "common.cuh"
+#include "dsa.h"
 
 namespace dsa {
 namespace {
@@ -434,7 +437,59 @@ compact_kernel(const uint32_t* __restrict__ bitmaps, int rows,
   }
 }
 
+// Stable rank of every row of head blockIdx.x by descending block count.
+// Row j's key is (len_j << 11) | (2047 - j), len_j clamped to [0, 2^20): the
+// keys of a head are distinct, and key_j > key_i exactly when row j has more
+// blocks than row i, or as many and a lower index, so
+//   rank(i) = #{j : key_j > key_i}
+// maps the head's rows one to one onto 0 .. nB-1 whatever row_ptr holds (a
+// malformed row_ptr only changes the lengths).  Every CTA of the head loads
+// all nB keys into shared memory (padded with -1 to a multiple of 4) and
+// ranks its own slice of the rows, one row per thread, reading the keys four
+// at a time (broadcast loads).
+__global__ void __launch_bounds__(1024)
+row_order_kernel(const int32_t* __restrict__ row_ptr, int nB, int per_cta,
+                 int32_t* __restrict__ order) {
+  __shared__ __align__(16) int key[DSA_MAX_BLOCKS];
+  const int bh = blockIdx.x;
+  const int32_t* rp = row_ptr + (size_t)bh * nB;
+  const int nB4 = (nB + 3) & ~3;
+  for (int j = threadIdx.x; j < nB4; j += blockDim.x) {
+    int k = -1;
+    if (j < nB) {
+      long long len = (long long)rp[j + 1] - rp[j];
+      len = len < 0 ? 0 : (len > (1 << 20) - 1 ? (1 << 20) - 1 : len);
+      k = (int)(len << 11) | (2047 - j);
+    }
+    key[j] = k;
+  }
+  __syncthreads();
+  const int i = blockIdx.y * per_cta + threadIdx.x;
+  if (threadIdx.x >= per_cta || i >= nB) return;
+  const int ki = key[i];
+  const int4* k4 = reinterpret_cast<const int4*>(key);
+  int rank = 0;
+  for (int j = 0; j < nB4 / 4; ++j) {
+    const int4 k = k4[j];
+    rank += (k.x > ki) + (k.y > ki) + (k.z > ki) + (k.w > ki);
+  }
+  order[(size_t)bh * nB + rank] = bh * nB + i;
+}
+
 }  // namespace
+
+cudaError_t launch_row_order(const int32_t* row_ptr, int BH, int nB, int num_sms, int32_t* order,
+                             cudaStream_t s) {
+  if (nB < 1 || nB > DSA_MAX_BLOCKS || BH < 1) return cudaErrorInvalidValue;
+  // enough CTAs for about two per SM, at least 64 rows each
+  int split = ceil_div(2 * (num_sms > 0 ? num_sms : 1), BH);
+  const int most = ceil_div(nB, 64);
+  split = split < 1 ? 1 : (split > most ? most : split);
+  const int per = ceil_div(nB, split);
+  const int threads = ceil_div(per, 32) * 32;  // <= 1024
+  row_order_kernel<<<dim3(BH, ceil_div(nB, per)), threads, 0, s>>>(row_ptr, nB, per, order);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_csr_scan(const int32_t* counts, int rows, int32_t* row_ptr, cudaStream_t s) {
   csr_scan_kernel<<<1, 1024, 0, s>>>(counts, rows, row_ptr);

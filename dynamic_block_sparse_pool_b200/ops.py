@@ -131,18 +131,40 @@ def select_topp(probs: torch.Tensor, p: float, cand: Optional[Csr] = None,
     return row_ptr, col_idx
 
 
+def row_order(row_ptr: torch.Tensor, B: int, H: int, nB: int,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """int32 [B*H*nB]: each head's rows by descending block count (ties by
+    row index), as global row indices; the order attn_fwd takes them in."""
+    rows = B * H * nB
+    if (row_ptr.dtype != torch.int32 or not row_ptr.is_cuda or not row_ptr.is_contiguous()
+            or row_ptr.numel() != rows + 1):
+        raise ValueError("row_ptr must be a contiguous int32 CUDA tensor of B*H*nB + 1 entries")
+    if out is None:
+        out = torch.empty(rows, device=row_ptr.device, dtype=torch.int32)
+    elif (out.dtype != torch.int32 or out.device != row_ptr.device or not out.is_contiguous()
+          or out.numel() != rows):
+        raise ValueError("out must be a contiguous int32 tensor of B*H*nB entries on row_ptr's device")
+    st = lib().dsa_row_order(row_ptr.data_ptr(), B, H, nB, out.data_ptr(), _stream(row_ptr))
+    check(st, "dsa_row_order")
+    return out
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.Tensor,
              col_idx: torch.Tensor, block: int, scale: Optional[float] = None,
              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
              blk_lse: Optional[torch.Tensor] = None, want_lse: bool = True,
-             want_blk_lse: bool = True):
+             want_blk_lse: bool = True, order: Optional[torch.Tensor] = None):
     """(O [B,H,N,D], lse [B,H,N] or None, blk_lse [nnz, block] or None).
 
-    When blk_lse is wanted but not given, nnz is read from row_ptr (one
-    device-to-host copy)."""
+    `order` (row_order's output) is the order in which the persistent CTAs
+    take the rows; it changes no output.  When blk_lse is wanted but not
+    given, nnz is read from row_ptr (one device-to-host copy)."""
     B, H, N, D = _check_qkv(q, k, v)
     nB = n_blocks(N, block)
     _check_csr((row_ptr, col_idx), B * H * nB)
+    if order is not None and (order.dtype != torch.int32 or order.device != q.device
+                              or not order.is_contiguous() or order.numel() != B * H * nB):
+        raise ValueError("order must be a contiguous int32 tensor of B*H*nB entries on q's device")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
@@ -152,8 +174,8 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.T
         nnz = int(row_ptr[-1].item())
         blk_lse = torch.empty(max(nnz, 1), block, device=q.device, dtype=torch.float32)
     st = lib().dsa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, N, D,
-                            block, scale, row_ptr.data_ptr(), col_idx.data_ptr(), out.data_ptr(),
-                            _ptr(lse), _ptr(blk_lse), _stream(q))
+                            block, scale, row_ptr.data_ptr(), col_idx.data_ptr(), _ptr(order),
+                            out.data_ptr(), _ptr(lse), _ptr(blk_lse), _stream(q))
     check(st, "dsa_attn_fwd")
     return out, lse, blk_lse
 
@@ -303,10 +325,13 @@ class SparseAttention(NamedTuple):
 def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: float,
                      block: int = 128, scale: Optional[float] = None,
                      cand: Optional[Csr] = None) -> SparseAttention:
-    """Whole pipeline: pooled scores -> Top-p selection -> sparse attention -> block mass."""
+    """Whole pipeline: pooled scores -> Top-p selection -> sparse attention
+    (rows taken longest first within each head) -> block mass."""
+    B, H, N, _ = q.shape
     probs = pool_score(q, k, block, scale, cand)
     row_ptr, col_idx = select_topp(probs, p, cand)
-    out, lse, blk = attn_fwd(q, k, v, row_ptr, col_idx, block, scale)
+    order = row_order(row_ptr, B, H, n_blocks(N, block))
+    out, lse, blk = attn_fwd(q, k, v, row_ptr, col_idx, block, scale, order=order)
     mass = block_mass(lse, blk, row_ptr, block)
     nnz = blk.shape[0] if int(row_ptr[-1].item()) > 0 else 0
     return SparseAttention(out, lse, probs, row_ptr, col_idx[:nnz], mass[:nnz])

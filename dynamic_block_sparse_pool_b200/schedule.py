@@ -124,8 +124,15 @@ class GsrsRunner:
                      torch.empty(cap, device=dev, dtype=torch.int32))
         self.later = (torch.empty(rows + 1, device=dev, dtype=torch.int32),
                       torch.empty(cap, device=dev, dtype=torch.int32))
+        # the order the attention takes each mask's rows in (longest first
+        # within each head)
+        self.base_order = torch.empty(rows, device=dev, dtype=torch.int32)
+        self.later_order = torch.empty(rows, device=dev, dtype=torch.int32)
         self.cur = None
         self.have_base = False
+
+    def _order_of(self, mask):
+        return self.base_order if mask is self.base else self.later_order
 
     def step(self, s: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> StepResult:
         kind, idx = self.kinds[s]
@@ -135,18 +142,20 @@ class GsrsRunner:
             return StepResult(kind, self.out, (self.all_rp, self.all_col), None, None)
         if kind == REUSE:
             ops.attn_fwd(q, k, v, self.cur[0], self.cur[1], self.block, self.scale, out=self.out,
-                         lse=self.lse, want_blk_lse=False)
+                         lse=self.lse, want_blk_lse=False, order=self._order_of(self.cur))
             return StepResult(kind, self.out, self.cur, None, None)
         # search: attention over the candidates with their exact block masses,
         # then Top-p on those masses within the candidates
         cand = self.base if self.have_base else (self.all_rp, self.all_col)
         ops.attn_fwd(q, k, v, cand[0], cand[1], self.block, self.scale, out=self.out,
-                     lse=self.lse, blk_lse=self.blk_lse)
+                     lse=self.lse, blk_lse=self.blk_lse,
+                     order=self._order_of(cand) if self.have_base else None)
         ops.block_mass(self.lse, self.blk_lse, cand[0], self.block, mass=self.mass)
         ops.mass_to_probs(cand[0], cand[1], self.mass, self.nB, out=self.probs)
         target = self.later if self.have_base else self.base
         ops.select_topp(self.probs, self.policy.p[idx], cand=cand, row_ptr=target[0],
                         col_idx=target[1], workspace=self.ws_sel)
+        ops.row_order(target[0], self.B, self.H, self.nB, out=self._order_of(target))
         self.have_base = True
         self.cur = target
         return StepResult(kind, self.out, cand, self.mass, target)

@@ -83,7 +83,7 @@ def test_exports_via_nm(lib):
 
 
 def test_version_and_workspace_sizes(lib):
-    assert lib.dsa_version() == 100
+    assert lib.dsa_version() == 200
     # pool: 2 * B*H*nB*D floats; select: B*H*nB*33 words
     assert lib.dsa_workspace_size(0, 1, 40, 75600, 128, 128) == 2 * 40 * 591 * 128 * 4
     assert lib.dsa_workspace_size(1, 1, 40, 75600, 128, 128) == 40 * 591 * 33 * 4
@@ -139,15 +139,28 @@ def test_select_rejects_sizes(lib):
 
 
 def test_attn_and_mass_reject(lib):
-    ok = (FAKE, FAKE, FAKE, 1, 1, 2, 256, 64, 128, 0.125, FAKE, FAKE, FAKE, None, None, None)
-    bad_out = ok[:12] + (FAKE + 8,) + ok[13:]
+    ok = (FAKE, FAKE, FAKE, 1, 1, 2, 256, 64, 128, 0.125, FAKE, FAKE, None, FAKE, None, None,
+          None)
+    bad_out = ok[:13] + (FAKE + 8,) + ok[14:]
     assert lib.dsa_attn_fwd(*bad_out) == _lib.DSA_ERR_INVALID_ARG
+    bad_order = ok[:12] + (FAKE + 2,) + ok[13:]
+    assert lib.dsa_attn_fwd(*bad_order) == _lib.DSA_ERR_INVALID_ARG
     no_v = ok[:2] + (None,) + ok[3:]
     assert lib.dsa_attn_fwd(*no_v) == _lib.DSA_ERR_INVALID_ARG
     bad_d = ok[:7] + (80,) + ok[8:]
     assert lib.dsa_attn_fwd(*bad_d) == _lib.DSA_ERR_INVALID_ARG
     assert lib.dsa_block_mass(None, FAKE, 1, 2, 256, 128, FAKE, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
     assert lib.dsa_block_mass(FAKE, FAKE, 1, 2, 256, 100, FAKE, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+
+
+def test_row_order_rejects(lib):
+    assert lib.dsa_row_order(None, 1, 2, 16, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_row_order(FAKE, 1, 2, 16, None, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_row_order(FAKE, 0, 2, 16, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_row_order(FAKE, 1, 2, 1025, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_row_order(FAKE, 1, 2, 0, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_row_order(FAKE + 2, 1, 2, 16, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_row_order(FAKE, 1 << 16, 1 << 10, 1024, FAKE, None) == _lib.DSA_ERR_INVALID_ARG
 
 
 def test_mass_to_probs_rejects(lib):
