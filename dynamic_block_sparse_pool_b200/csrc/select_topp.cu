@@ -444,9 +444,10 @@ compact_kernel(const uint32_t* __restrict__ bitmaps, int rows,
 //   rank(i) = #{j : key_j > key_i}
 // maps the head's rows one to one onto 0 .. nB-1 whatever row_ptr holds (a
 // malformed row_ptr only changes the lengths).  Every CTA of the head loads
-// all nB keys into shared memory (padded with -1 to a multiple of 4) and
-// ranks its own slice of the rows, one row per thread, reading the keys four
-// at a time (broadcast loads).
+// all nB keys into shared memory (padded with -1 to a multiple of 4; at
+// least 256 threads, so the loads take a few rounds) and ranks its own
+// slice of the rows, one row per thread, reading the keys four at a time
+// (broadcast loads).
 __global__ void __launch_bounds__(1024)
 row_order_kernel(const int32_t* __restrict__ row_ptr, int nB, int per_cta,
                  int32_t* __restrict__ order) {
@@ -469,6 +470,7 @@ row_order_kernel(const int32_t* __restrict__ row_ptr, int nB, int per_cta,
   const int ki = key[i];
   const int4* k4 = reinterpret_cast<const int4*>(key);
   int rank = 0;
+#pragma unroll 4
   for (int j = 0; j < nB4 / 4; ++j) {
     const int4 k = k4[j];
     rank += (k.x > ki) + (k.y > ki) + (k.z > ki) + (k.w > ki);
@@ -486,7 +488,7 @@ cudaError_t launch_row_order(const int32_t* row_ptr, int BH, int nB, int num_sms
   const int most = ceil_div(nB, 64);
   split = split < 1 ? 1 : (split > most ? most : split);
   const int per = ceil_div(nB, split);
-  const int threads = ceil_div(per, 32) * 32;  // <= 1024
+  const int threads = per > 256 ? ceil_div(per, 32) * 32 : 256;  // <= 1024
   row_order_kernel<<<dim3(BH, ceil_div(nB, per)), threads, 0, s>>>(row_ptr, nB, per, order);
   return cudaGetLastError();
 }
