@@ -28,8 +28,9 @@ SIGNATURES = {
     "dsa_pool_score": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_select_topp": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_row_order": (_i, [_vp, _i, _i, _i, _vp, _vp]),
-    "dsa_attn_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp,
-                          _vp]),
+    "dsa_attn_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "dsa_attn_fwd_ordered": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp,
+                                  _vp, _vp, _vp]),
     "dsa_block_mass": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "dsa_attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
                           _vp, _vp, _vp, _vp, _sz, _vp]),

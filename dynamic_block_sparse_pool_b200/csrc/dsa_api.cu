@@ -204,7 +204,7 @@ size_t bwd_ws_bytes(long long BH, long long nB, long long N) {
 
 extern "C" {
 
-int dsa_version(void) { return 200; }
+int dsa_version(void) { return 101; }
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
@@ -337,8 +337,17 @@ dsa_status dsa_row_order(const int32_t* row_ptr, int B, int H, int nB, int32_t* 
 
 dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype dt, int B, int H,
                         int N, int D, int block, float scale, const int32_t* row_ptr,
-                        const int32_t* col_idx, const int32_t* row_order, void* out, float* lse,
-                        float* blk_lse, void* stream) {
+                        const int32_t* col_idx, void* out, float* lse, float* blk_lse,
+                        void* stream) {
+  return dsa_attn_fwd_ordered(q, k, v, dt, B, H, N, D, block, scale, row_ptr, col_idx, nullptr,
+                              out, lse, blk_lse, stream);
+}
+
+dsa_status dsa_attn_fwd_ordered(const void* q, const void* k, const void* v, dsa_dtype dt, int B,
+                                int H, int N, int D, int block, float scale,
+                                const int32_t* row_ptr, const int32_t* col_idx,
+                                const int32_t* row_order, void* out, float* lse, float* blk_lse,
+                                void* stream) {
   g_last_error.clear();
   if (!q || !k || !v || !out || !row_ptr || !col_idx)
     return fail(DSA_ERR_INVALID_ARG, "null q, k, v, out, row_ptr or col_idx");
@@ -587,8 +596,9 @@ dsa_status dsa_sparse_attention_host(const void* q, const void* k, const void* v
         (st = dsa_select_topp(probs, rows, (int)nB, p, nullptr, nullptr, rp, ci_idx,
                               slot + L.ws_sel, L.sel_bytes, h.s_comp)) != DSA_OK ||
         (st = dsa_row_order(rp, 1, hn, (int)nB, order, h.s_comp)) != DSA_OK ||
-        (st = dsa_attn_fwd(slot + L.q, slot + L.k, slot + L.v, dt, 1, hn, N, D, block, scale, rp,
-                           ci_idx, order, slot + L.out, lse, bl, h.s_comp)) != DSA_OK ||
+        (st = dsa_attn_fwd_ordered(slot + L.q, slot + L.k, slot + L.v, dt, 1, hn, N, D, block,
+                                   scale, rp, ci_idx, order, slot + L.out, lse, bl,
+                                   h.s_comp)) != DSA_OK ||
         (st = dsa_block_mass(lse, bl, 1, hn, N, block, rp, reinterpret_cast<float*>(slot + L.mass),
                              h.s_comp)) != DSA_OK)
       return st;  // the inner call set the message

@@ -156,9 +156,11 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.T
              want_blk_lse: bool = True, order: Optional[torch.Tensor] = None):
     """(O [B,H,N,D], lse [B,H,N] or None, blk_lse [nnz, block] or None).
 
-    `order` (row_order's output) is the order in which the persistent CTAs
-    take the rows; it changes no output.  When blk_lse is wanted but not
-    given, nnz is read from row_ptr (one device-to-host copy)."""
+    Without `order` this is dsa_attn_fwd (rows in index order); with it,
+    dsa_attn_fwd_ordered: `order` (row_order's output) is the order in which
+    the persistent CTAs take the rows, and changes no output.  When blk_lse
+    is wanted but not given, nnz is read from row_ptr (one device-to-host
+    copy)."""
     B, H, N, D = _check_qkv(q, k, v)
     nB = n_blocks(N, block)
     _check_csr((row_ptr, col_idx), B * H * nB)
@@ -173,10 +175,17 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.T
     if want_blk_lse and blk_lse is None:
         nnz = int(row_ptr[-1].item())
         blk_lse = torch.empty(max(nnz, 1), block, device=q.device, dtype=torch.float32)
-    st = lib().dsa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, N, D,
-                            block, scale, row_ptr.data_ptr(), col_idx.data_ptr(), _ptr(order),
-                            out.data_ptr(), _ptr(lse), _ptr(blk_lse), _stream(q))
-    check(st, "dsa_attn_fwd")
+    if order is None:
+        st = lib().dsa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, N,
+                                D, block, scale, row_ptr.data_ptr(), col_idx.data_ptr(),
+                                out.data_ptr(), _ptr(lse), _ptr(blk_lse), _stream(q))
+        check(st, "dsa_attn_fwd")
+    else:
+        st = lib().dsa_attn_fwd_ordered(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B,
+                                        H, N, D, block, scale, row_ptr.data_ptr(),
+                                        col_idx.data_ptr(), order.data_ptr(), out.data_ptr(),
+                                        _ptr(lse), _ptr(blk_lse), _stream(q))
+        check(st, "dsa_attn_fwd_ordered")
     return out, lse, blk_lse
 
 

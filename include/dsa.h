@@ -10,10 +10,11 @@
  *                    blocks or over a candidate set C_i (reduced search).
  *   dsa_select_topp  per row i: the shortest prefix of the candidates ordered
  *                    by (P desc, block index asc) whose mass is >= p, as CSR.
- *   dsa_row_order    the order in which dsa_attn_fwd takes a mask's rows
- *                    (each head's longest first).
+ *   dsa_row_order    the order in which the attention takes a mask's rows
+ *                    (each head's longest first), for dsa_attn_fwd_ordered.
  *   dsa_attn_fwd     exact softmax attention of every query in B_i over the
- *                    keys of the selected blocks, with per-block log-sums.
+ *                    keys of the selected blocks, with per-block log-sums
+ *                    (dsa_attn_fwd_ordered: the same, rows in a given order).
  *   dsa_block_mass   the exact softmax mass each selected block receives.
  *   dsa_attn_bwd     gradients of the attention for a fixed mask.
  *   dsa_mass_to_probs  those masses as dense rows, for a Top-p selection on
@@ -176,7 +177,7 @@ dsa_status dsa_select_topp(const float* probs, int rows, int nB, float p,
                            void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * The order in which dsa_attn_fwd's persistent CTAs take a mask's rows (DSV
+ * The order in which the attention's persistent CTAs take a mask's rows (DSV
  * abstract: the work per query block is skewed, and handed out
  * dynamically).  The CTAs draw rows one at a time, each as soon as it is
  * free; the launch ends when the last CTA finishes, so the rows drawn last
@@ -192,8 +193,9 @@ dsa_status dsa_select_topp(const float* probs, int rows, int nB, float p,
  *   order     device out, int32 [B*H*nB]: a permutation of 0 .. B*H*nB-1
  *             whatever row_ptr holds (a malformed row_ptr only makes the
  *             order arbitrary).
- * One launch, one CTA per head, nB^2 comparisons per head (nB = 591: a few
- * microseconds).  Limits: nB <= DSA_MAX_BLOCKS.
+ * One launch of a few CTAs per head (about two per SM in all), nB^2
+ * comparisons per head (40 heads of nB = 591: under 10 microseconds).
+ * Limits: nB <= DSA_MAX_BLOCKS.
  */
 dsa_status dsa_row_order(const int32_t* row_ptr, int B, int H, int nB, int32_t* order,
                          void* stream);
@@ -209,12 +211,6 @@ dsa_status dsa_row_order(const int32_t* row_ptr, int B, int H, int nB, int32_t* 
  *
  *   q, k, v   [B, H, N, D] in dt.   out: [B, H, N, D] in dt.
  *   row_ptr, col_idx   CSR block mask over the B*H*nB rows (any column order).
- *   row_order optional, int32 [B*H*nB]: a permutation of the row indices,
- *             the order in which the persistent CTAs take the rows
- *             (dsa_row_order writes one); NULL takes them in index order.
- *             It changes only which CTA computes a row and when: every
- *             output is the same with any order.  The fp32 / block-64 path
- *             ignores it.
  *   lse       optional out, fp32 [B, H, N]: natural-log sum of exp(scale q.k)
  *             over the attended keys; -inf for a row with no blocks.
  *   blk_lse   optional out, fp32 [nnz, block]: blk_lse[s*block + t'] =
@@ -228,24 +224,42 @@ dsa_status dsa_row_order(const int32_t* row_ptr, int B, int H, int nB, int32_t* 
  * ticket counter in device memory that the library keeps per device (4,096
  * counters used in rotation, one per launch; the launch's last CTA zeroes its
  * counter again), so rows of skewed length are balanced dynamically (DSV
- * abstract); each head's rows longest first (dsa_row_order) leave the short
- * rows for the end of the launch, where they fill the gaps that the last
- * long rows leave.  Launches that run at the same time, on any streams, use
+ * abstract); this call takes them in index order, dsa_attn_fwd_ordered in a
+ * given one.  Launches that run at the same time, on any streams, use
  * different counters while fewer than 4,096 launches lie between them; a
  * captured CUDA graph replays its launch with the counter of its capture.
  * Errors: a malformed row (column index outside [0, nB), decreasing row_ptr)
- * sets the device error word and is written as an empty row; a row_order
- * entry outside [0, B*H*nB) sets it and is passed over (a row that a
- * non-permutation leaves out is not written; one it names twice is
- * written twice, with the same values); a device wait
+ * sets the device error word and is written as an empty row; a device wait
  * that runs out (1 s) sets the error word and leaves the rows that the
  * affected CTA had not finished unwritten.  dsa_device_status reports both.
  */
 dsa_status dsa_attn_fwd(const void* q, const void* k, const void* v, dsa_dtype dt,
                         int B, int H, int N, int D, int block, float scale,
                         const int32_t* row_ptr, const int32_t* col_idx,
-                        const int32_t* row_order, void* out, float* lse, float* blk_lse,
-                        void* stream);
+                        void* out, float* lse, float* blk_lse, void* stream);
+
+/*
+ * dsa_attn_fwd with the rows taken in a given order (DSV abstract: skewed
+ * work per query block).  The persistent CTAs draw tickets 0, 1, 2, ...;
+ * ticket t is row row_order[t].  With each head's rows longest first
+ * (dsa_row_order) the short rows come at the end of the launch, where they
+ * fill the gaps that the last long rows leave.
+ *
+ *   row_order optional, device, int32 [B*H*nB]: a permutation of the row
+ *             indices; NULL takes them in index order (= dsa_attn_fwd).
+ *   the other arguments as for dsa_attn_fwd.
+ * The order changes only which CTA computes a row and when: every output is
+ * the same with any order.  The fp32 / block-64 path ignores it.
+ * Errors as for dsa_attn_fwd, and: a row_order entry outside [0, B*H*nB)
+ * sets the device error word and is passed over (a row that a
+ * non-permutation leaves out is not written; one it names twice is written
+ * twice, with the same values).
+ */
+dsa_status dsa_attn_fwd_ordered(const void* q, const void* k, const void* v, dsa_dtype dt,
+                                int B, int H, int N, int D, int block, float scale,
+                                const int32_t* row_ptr, const int32_t* col_idx,
+                                const int32_t* row_order, void* out, float* lse,
+                                float* blk_lse, void* stream);
 
 /*
  * Gradients of dsa_attn_fwd's O for a fixed mask (DSV abstract: DiTs are
@@ -291,7 +305,7 @@ dsa_status dsa_block_mass(const float* lse, const float* blk_lse,
 
 /*
  * The whole pipeline (dsa_pool_score, dsa_select_topp, dsa_row_order,
- * dsa_attn_fwd with that order, dsa_block_mass; full search, Top-p
+ * dsa_attn_fwd_ordered with that order, dsa_block_mass; full search, Top-p
  * threshold p) on HOST-resident Q, K,
  * V, with O written back to host memory.  Every (b, h) is an independent
  * problem (DSV abstract: each head is its own work item), so the B*H axis is

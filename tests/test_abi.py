@@ -83,7 +83,7 @@ def test_exports_via_nm(lib):
 
 
 def test_version_and_workspace_sizes(lib):
-    assert lib.dsa_version() == 200
+    assert lib.dsa_version() == 101
     # pool: 2 * B*H*nB*D floats; select: B*H*nB*33 words
     assert lib.dsa_workspace_size(0, 1, 40, 75600, 128, 128) == 2 * 40 * 591 * 128 * 4
     assert lib.dsa_workspace_size(1, 1, 40, 75600, 128, 128) == 40 * 591 * 33 * 4
@@ -139,12 +139,17 @@ def test_select_rejects_sizes(lib):
 
 
 def test_attn_and_mass_reject(lib):
-    ok = (FAKE, FAKE, FAKE, 1, 1, 2, 256, 64, 128, 0.125, FAKE, FAKE, None, FAKE, None, None,
-          None)
-    bad_out = ok[:13] + (FAKE + 8,) + ok[14:]
+    ok = (FAKE, FAKE, FAKE, 1, 1, 2, 256, 64, 128, 0.125, FAKE, FAKE, FAKE, None, None, None)
+    bad_out = ok[:12] + (FAKE + 8,) + ok[13:]
     assert lib.dsa_attn_fwd(*bad_out) == _lib.DSA_ERR_INVALID_ARG
-    bad_order = ok[:12] + (FAKE + 2,) + ok[13:]
-    assert lib.dsa_attn_fwd(*bad_order) == _lib.DSA_ERR_INVALID_ARG
+    # the ordered entry: the order after col_idx, the rest as above
+    ordered = ok[:12] + (FAKE,) + ok[12:]
+    assert lib.dsa_attn_fwd_ordered(*(ordered[:12] + (FAKE + 2,) + ordered[13:])) == \
+        _lib.DSA_ERR_INVALID_ARG                                                      # order
+    assert "aligned" in lib.dsa_last_error().decode()
+    assert lib.dsa_attn_fwd_ordered(*(ordered[:13] + (FAKE + 8,) + ordered[14:])) == \
+        _lib.DSA_ERR_INVALID_ARG                                                      # out
+    assert lib.dsa_attn_fwd_ordered(*(ordered[:7] + (80,) + ordered[8:])) == _lib.DSA_ERR_INVALID_ARG
     no_v = ok[:2] + (None,) + ok[3:]
     assert lib.dsa_attn_fwd(*no_v) == _lib.DSA_ERR_INVALID_ARG
     bad_d = ok[:7] + (80,) + ok[8:]
